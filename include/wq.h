@@ -1,0 +1,184 @@
+/*
+ * wq.h - C ABI of the weight-only-quantized decode linear for NVIDIA B200 (sm_100a).
+ *
+ *   y[M, N] = x[M, K] . deq(W)[N, K]^T      x, y bf16; W stored at reduced width,
+ *                                           dequantized inside the kernel; fp32 accumulation.
+ *
+ * The operation is the linear layer of autoregressive decode whose weight stream
+ * bounds each step: gpt-fast write-up (m.greenbasetech.com article
+ * 46368139_1106049486), paragraphs on the memory-bandwidth bound and on int8 /
+ * int4 weight-only quantization; FP6-LLM / TC-FPx article (m.zhengruan.com news
+ * 124379), section "重新设计内核方案" (dequantization fused with the matrix multiply
+ * in one kernel, weights prepacked before inference).
+ *
+ * Conventions for every call:
+ *   - Every function returns a wq_status; on failure wq_last_error() returns a
+ *     thread-local message.  Argument errors are detected on the host before any
+ *     CUDA call or launch, so a rejected call has no side effect.
+ *   - The caller owns every buffer.  No call keeps a pointer after it returns
+ *     (device work queued by wq_linear / wq_unpack_debug reads its buffers until it
+ *     completes on the given stream).
+ *   - "host" pointers are ordinary CPU memory; "device" pointers are CUDA global
+ *     memory of the current device, 16-byte aligned (checked: WQ_ERR_ALIGN).
+ *   - Matrices are row-major.  Scales and zeros are passed as raw 16-bit patterns
+ *     (uint16_t): fp16 for int8 and FP6, bf16 for int4.
+ *   - Shapes: N >= 0, M in [0, 32], K >= 0 with K % 64 == 0; int4 also needs a
+ *     group size g in {32, 64, 128} with K % g == 0.  M == 0 or N == 0 is a no-op.
+ *     K == 0 writes y = 0 (empty sum).
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Weight formats. */
+typedef enum {
+  WQ_INT8 = 0,     /* W8A16: int8 codes, one fp16 scale per output channel (row n) */
+  WQ_INT4 = 1,     /* W4A16: uint4 codes, bf16 scale + bf16 zero per group of g along K */
+  WQ_FP6_E3M2 = 2, /* W6A16: FP6 e3m2 codes, one fp16 scale per output channel, 2+4-bit planes */
+  WQ_BF16 = 3      /* unquantized bf16 weights (the reference kernel), no scales */
+} wq_fmt;
+
+typedef enum {
+  WQ_OK = 0,
+  WQ_ERR_NULL = 1,    /* a required pointer is NULL, or a forbidden one is not */
+  WQ_ERR_SHAPE = 2,   /* M, N or K outside the supported set */
+  WQ_ERR_FMT = 3,     /* unknown format */
+  WQ_ERR_GROUP = 4,   /* int4 group size not in {32, 64, 128} or not dividing K */
+  WQ_ERR_ALIGN = 5,   /* a device pointer is not 16-byte aligned */
+  WQ_ERR_CUDA = 6,    /* a CUDA runtime call or launch failed (message has the CUDA error) */
+  WQ_ERR_RANGE = 7,   /* quantizer input non-finite, a code out of range, or a scale overflows */
+  WQ_ERR_TIMEOUT = 8  /* a bounded device-side wait gave up (reported by wq_sync_status) */
+} wq_status;
+
+/* ------------------------------------------------------------------ sizes */
+
+/* Bytes of the packed weight buffer for an N x K matrix in `fmt`
+ * (int8: N*K; int4: N*K/2; FP6: 3*N*K/4 = N*K/4 (2-bit plane) + N*K/2 (4-bit plane);
+ * bf16: 2*N*K).  Returns 0 for an unknown format or a negative size. */
+size_t wq_packed_size(int fmt, int64_t N, int64_t K);
+
+/* Bytes of the scale buffer (and, for int4, of the equally sized zero buffer):
+ * int8 / FP6: 2*N (fp16 per row); int4: 2*N*(K/g) (bf16 per row and group);
+ * bf16: 0.  Returns 0 for an invalid format or group size. */
+size_t wq_scales_size(int fmt, int64_t N, int64_t K, int groupsize);
+
+/* ------------------------------------------------------------ quantizers
+ * Offline, host -> host.  W is float32 [N, K] row-major.  All arithmetic is in
+ * float64 on the float32 values; rounding of scales and zeros as stated.
+ * A non-finite weight or an overflowing scale gives WQ_ERR_RANGE.          */
+
+/* int8, symmetric per output channel (gpt-fast write-up, paragraph on int8
+ * weight-only quantization):  s_n = fp16_RNE(max_k |W[n,k]| / 127),
+ * q = clamp(RNE(W / s_n), -127, 127); s_n == 0 gives q == 0.
+ * q: int8 [N, K] (host); s_fp16: uint16 [N] (host). */
+wq_status wq_quantize_int8(const float* W, int64_t N, int64_t K, int8_t* q, uint16_t* s_fp16);
+
+/* int4, asymmetric, grouped along K (gpt-fast write-up, paragraph on int4 with
+ * group-wise quantization; gpt-fast guide, section "量化技术深度解析", groupsize 32):
+ * per group of g consecutive k of row n, z = bf16 rounded down from min W,
+ * s = bf16 rounded up from (max W - z) / 15, q = clamp(RNE((W - z) / s), 0, 15),
+ * deq = q * s + z.  q: uint8 [N, K] one code 0..15 per byte (host);
+ * s_bf16, z_bf16: uint16 [N, K/g] (host). */
+wq_status wq_quantize_int4(const float* W, int64_t N, int64_t K, int groupsize, uint8_t* q,
+                           uint16_t* s_bf16, uint16_t* z_bf16);
+
+/* FP6 e3m2 per output channel (FP6-LLM / TC-FPx article, opening sections and
+ * "重新设计内核方案"): codes 0..63 with bit 5 sign, bits 4..2 exponent (bias 3),
+ * bits 1..0 mantissa, subnormals at exponent 0, no inf/nan, max 28.
+ * s_n = fp16_RNE(max |W[n,:]| / 28); code = e3m2 value nearest W / s_n, ties to the
+ * even code, saturating at +-28; magnitudes rounding to zero give code 0.
+ * code: uint8 [N, K] (host); s_fp16: uint16 [N] (host). */
+wq_status wq_quantize_fp6(const float* W, int64_t N, int64_t K, uint8_t* code, uint16_t* s_fp16);
+
+/* ---------------------------------------------------------------- packers
+ * Offline, host -> host, run before inference (FP6-LLM / TC-FPx article,
+ * "重新设计内核方案": bit-level prepacking reorganises the weights before inference
+ * so that they are fetched as aligned 32/64-bit and wider blocks).  Every packed
+ * row is a whole number of 16-byte units, so a warp reads 512 contiguous bytes
+ * per 128-bit load and a row-major 2-D TMA box can stage any tile.
+ * Packed buffers are host byte arrays; copy them to the device as they are.      */
+
+/* int8: packed[n*K + k] = (uint8)(q[n,k] + 128) (offset binary).
+ * q: int8 [N, K] in [-127, 127] (host); packed: wq_packed_size(WQ_INT8) bytes (host). */
+wq_status wq_pack_int8(const int8_t* q, int64_t N, int64_t K, void* packed);
+
+/* int4: byte n*K/2 + k/2 holds q[n,k] in its low nibble for even k, high nibble
+ * for odd k.  q: uint8 [N, K] codes 0..15 (host); packed: N*K/2 bytes (host). */
+wq_status wq_pack_int4(const uint8_t* q, int64_t N, int64_t K, void* packed);
+
+/* FP6: each code c (bit 5 sign, bits 4..2 exponent e2 e1 e0, bits 1..0 mantissa)
+ * is split into a 2-bit piece (sign, e2) and a 4-bit piece c & 0xF = (e1 e0 m1 m0)
+ * - the 2+4 split of FP6-LLM / TC-FPx, "重新设计内核方案" - stored in two planes:
+ * the 2-bit plane first (N*K/4 bytes, row n at byte n*K/4), then the 4-bit plane
+ * (N*K/2 bytes).  Bit positions are taken
+ * modulo 32 inside little-endian 32-bit words.
+ *   4-bit plane: word t of row n (bytes n*K/2 + 4t .. +3) holds k = 8t + i,
+ *     i = j + 4h (j in 0..3, h in 0..1); bit b (0..3) of the piece of k sits at
+ *     bit (5 + 16h - 4j + b) mod 32.
+ *   2-bit plane: word u of row n (bytes n*K/4 + 4u .. +3) holds k = 16u + i,
+ *     i = 8c + j + 4h (c, h in 0..1, j in 0..3); with T = {0,1,4,5,8,9,12,13}[4c + j]
+ *     the sign bit sits at (15 + 16h - T) mod 32 and e2 at (9 + 16h - T) mod 32.
+ * With this permutation the kernel forms the bf16 pair (k = 8t+j, 8t+j+4) as
+ * (rotl(P4, 4j) & 0x01E001E0) | (rotl(P2, T) & 0x82008200): sign at bit 15,
+ * exponent field = e, mantissa = m/4, i.e. the code value times 2^-124
+ * (e = 0 codes land on bf16 subnormals).
+ * code: uint8 [N, K] codes 0..63 (host); packed: 3*N*K/4 bytes (host). */
+wq_status wq_prepack_fp6(const uint8_t* code, int64_t N, int64_t K, void* packed);
+
+/* ---------------------------------------------------------------- compute */
+
+/* y = x . deq(W)^T on the GPU, asynchronously on `cuda_stream` (a cudaStream_t;
+ * NULL = legacy default stream).
+ *   x:      device bf16 [M, K]
+ *   packed: device, layout of the packer for `fmt` (bf16: plain [N, K] bf16)
+ *   scales: device uint16 per wq_scales_size (NULL for WQ_BF16)
+ *   zeros:  device bf16 [N, K/g] for WQ_INT4, must be NULL otherwise
+ *   y:      device bf16 [M, N], written with round-to-nearest-even
+ * M in [0, 32].  Dispatch: M <= 4 runs the CUDA-core split-K GEMV; larger M runs
+ * the tensor-core (tcgen05) swap-AB GEMM where built.  Launch errors give
+ * WQ_ERR_CUDA.  Buffers must not overlap y. */
+wq_status wq_linear(const void* x, const void* packed, const void* scales, const void* zeros,
+                    void* y, int64_t M, int64_t N, int64_t K, int fmt, int groupsize,
+                    void* cuda_stream);
+
+/* Launch-option flags for wq_linear_ex. */
+#define WQ_LAUNCH_PDL 0x1u /* programmatic dependent launch: the kernel may start
+                              streaming weights while the previous kernel on the stream
+                              is still running.  The caller guarantees that packed,
+                              scales and zeros are not written by any work still in
+                              flight on the stream; x is read and y written only after
+                              the previous kernel has completed. */
+
+/* wq_linear with launch-option flags (0 = exactly wq_linear). */
+wq_status wq_linear_ex(const void* x, const void* packed, const void* scales, const void* zeros,
+                       void* y, int64_t M, int64_t N, int64_t K, int fmt, int groupsize,
+                       void* cuda_stream, unsigned flags);
+
+/* Test support: run the kernels' own weight decode on the GPU and write, for
+ * every (n, k), the decoded code value (int8 q, int4 q, FP6 e3m2 value, bf16 W)
+ * as bf16 - all exactly representable - to out_bf16 [N, K] (device).  No scale
+ * or zero is applied.  Asynchronous on cuda_stream. */
+wq_status wq_unpack_debug(const void* packed, int fmt, int64_t N, int64_t K, void* out_bf16,
+                          void* cuda_stream);
+
+/* Synchronizes the stream and reports WQ_ERR_CUDA for a pending asynchronous
+ * error, WQ_ERR_TIMEOUT if a bounded device wait expired since the last call. */
+wq_status wq_sync_status(void* cuda_stream);
+
+/* Thread-local message for the last failing call of this thread ("" if none). */
+const char* wq_last_error(void);
+
+/* Library version string, e.g. "wq 0.1 sm_100a". */
+const char* wq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

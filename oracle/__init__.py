@@ -1,0 +1,34 @@
+"""Plain, slow, obviously-correct CPU oracle for the weight-only-quantized decode linear.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` may import anything from this
+package.  The product path (``gemm_wq_linear_b200``) never imports it and shares
+no code, table or constant generator with it.
+
+What it computes (all arithmetic in float64 unless a format fixes a precision):
+
+* ``rounding``  - round-to-nearest-even and directed rounding onto fp16 / bf16,
+                  written from the IEEE-754 definition of a binary format.
+* ``formats``   - the three weight formats: int8 with a per-output-channel fp16
+                  scale (W8A16), int4 grouped along K with a bf16 scale and zero
+                  per group (W4A16), FP6 e3m2 with a per-output-channel fp16 scale
+                  (W6A16); quantizers, code decoders and dequantizers.
+* ``layout``    - unpackers for the packed byte layouts, written from the layout
+                  definition (the library's packers are checked against them).
+* ``linear``    - ``y = x . deq(W)^T`` in float64 and its bf16 rounding.
+
+Sources (cited by page and section, never by any other handle):
+
+* gpt-fast write-up, m.greenbasetech.com article 46368139_1106049486 -
+  paragraphs on int8 weight-only quantization and on int4 with group-wise
+  quantization (group size 32).
+* gpt-fast guide, jsqmd.com news 1295739 - section "量化技术深度解析"
+  (quantization deep dive): ``quantize.py --mode int4 --groupsize 32``.
+* FP6-LLM / TC-FPx article, m.zhengruan.com news 124379 - section
+  "重新设计内核方案" (redesigning the kernel): FP6 weights, fused dequant + matmul,
+  bit-level prepacking, 2+4 weight splitting.
+
+Parity status of each function is stated in its docstring ("pinned by ...").
+"""
+
+from . import rounding, formats, layout, linear  # noqa: F401

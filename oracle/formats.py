@@ -1,0 +1,178 @@
+"""Weight formats of the decode linear: quantize, decode codes, dequantize.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).  float64 throughout; the
+storage precisions (fp16 / bf16 scales and zeros) are fixed by the formats.
+
+Sources:
+
+* int8 weight-only, one scale per output channel: gpt-fast write-up
+  (m.greenbasetech.com article 46368139_1106049486), paragraph introducing int8
+  weight quantization to cut the bytes loaded per parameter.
+* int4 grouped along K with scale and zero per group, group size 32: same
+  write-up, paragraph on int4 + group-wise quantization; gpt-fast guide
+  (jsqmd.com news 1295739), section "量化技术深度解析", ``--mode int4 --groupsize 32``.
+* FP6 weights with 16-bit activations (W6A16), split of each 6-bit weight into
+  a 2-bit and a 4-bit piece: FP6-LLM / TC-FPx article (m.zhengruan.com news
+  124379), section "重新设计内核方案".
+
+Readings of what the pages leave open:
+
+* int8: symmetric, s_n = fp16_RNE(max_k |W[n,k]| / 127),
+  q = clamp(RNE(W / s_n), -127, 127), deq = s_n * q.  s_n == 0 gives q == 0.
+* int4: unsigned codes 0..15 with a float offset zero: for each group of g
+  consecutive k of row n, z = bf16_round_down(min W), s = bf16_round_up((max W - z)/15),
+  q = clamp(RNE((W - z)/s), 0, 15), deq = q*s + z.  Directed rounding keeps every
+  weight inside [z, z + 15 s], so |W - deq| <= s/2 holds for every element.
+  s == 0 gives q == 0 (deq == z).
+* FP6 e3m2: bit 5 sign, bits 4..2 exponent e (bias 3), bits 1..0 mantissa m;
+  |v| = 2**(e-3) * (1 + m/4) for e > 0 and 2**-2 * (m/4) for e == 0; no inf/nan,
+  max 28, smallest nonzero 1/16.  s_n = fp16_RNE(max|W[n,:]| / 28); the code is
+  the e3m2 value nearest to W/s_n (ties to the even code, i.e. even mantissa),
+  saturating at +-28; a magnitude that rounds to zero takes code 0x00.
+* All quotients are float64 divisions of the float32 weight values.
+"""
+
+import numpy as np
+
+from .rounding import fp16_rne, bf16_down, bf16_up
+
+INT8_QMAX = 127
+INT4_QMAX = 15
+FP6_MAX = 28.0
+
+
+# --------------------------------------------------------------------- FP6 e3m2
+def e3m2_value(code):
+    """Real value of FP6 e3m2 codes (ints 0..63), straight from the definition.
+
+    Pinned by a hand-listed table of the 32 magnitudes, max 28, smallest
+    nonzero 1/16, sign symmetry and monotonicity (tests/test_oracle.py).
+    """
+    code = np.asarray(code, dtype=np.int64)
+    if np.any((code < 0) | (code > 63)):
+        raise ValueError("FP6 code out of range")
+    s = (code >> 5) & 1
+    e = (code >> 2) & 7
+    m = code & 3
+    mag = np.where(e > 0, np.ldexp(1.0 + m / 4.0, e - 3), np.ldexp(m / 4.0, -2))
+    return np.where(s == 1, -mag, mag).astype(np.float64)
+
+
+def _e3m2_round(r):
+    """Nearest e3m2 code to float64 ``r`` (ties to even code), saturating at 28.
+
+    The 32 magnitudes increase with the code, so the two candidates around |r|
+    are found by a sorted search; the closer one wins, and on an exact tie the
+    one with the even code (even mantissa) wins.  Above 28 the only candidate
+    is 28.
+    """
+    r = np.asarray(r, dtype=np.float64)
+    mags = e3m2_value(np.arange(32))
+    a = np.abs(r)
+    hi = np.clip(np.searchsorted(mags, a, side="left"), 0, 31)  # mags[hi] >= a (or hi == 31)
+    lo = np.clip(hi - 1, 0, 31)
+    d_lo = np.abs(a - mags[lo])
+    d_hi = np.abs(mags[hi] - a)
+    best = np.where(d_lo < d_hi, lo, hi)
+    best = np.where((d_lo == d_hi) & (lo != hi), np.where(lo % 2 == 0, lo, hi), best)
+    sign = (r < 0) & (best != 0)
+    return (best + 32 * sign).astype(np.uint8)
+
+
+def quantize_fp6(W):
+    """W float32 [N, K] -> (codes uint8 [N, K] in 0..63, scale bits uint16 [N] fp16).
+
+    Pinned by: every |W/s - v(code)| is at most half the local e3m2 spacing,
+    saturation at 28, hand-computed rows (tests/golden), ties to even.
+    """
+    W = np.asarray(W, dtype=np.float32).astype(np.float64)
+    _check_finite(W)
+    amax = np.max(np.abs(W), axis=1) if W.shape[1] else np.zeros(W.shape[0])
+    s = fp16_rne(amax / FP6_MAX)
+    if np.any(np.isinf(s)):
+        raise ValueError("fp16 scale overflow")
+    safe = np.where(s == 0, 1.0, s)
+    codes = _e3m2_round(W / safe[:, None])
+    codes = np.where(s[:, None] == 0, 0, codes).astype(np.uint8)
+    return codes, _fp16_bits(s)
+
+
+def dequant_fp6(codes, s_bits):
+    from .rounding import fp16_value
+    s = fp16_value(s_bits)
+    return e3m2_value(codes) * s[:, None]
+
+
+# --------------------------------------------------------------------- int8
+def quantize_int8(W):
+    """W float32 [N, K] -> (q int8 [N, K] in -127..127, scale bits uint16 [N] fp16).
+
+    Pinned by: |W - s q| <= s/2 per element, q range, hand-computed rows.
+    """
+    W = np.asarray(W, dtype=np.float32).astype(np.float64)
+    _check_finite(W)
+    amax = np.max(np.abs(W), axis=1) if W.shape[1] else np.zeros(W.shape[0])
+    s = fp16_rne(amax / INT8_QMAX)
+    if np.any(np.isinf(s)):
+        raise ValueError("fp16 scale overflow")
+    safe = np.where(s == 0, 1.0, s)
+    q = np.clip(np.rint(W / safe[:, None]), -INT8_QMAX, INT8_QMAX)
+    q = np.where(s[:, None] == 0, 0, q).astype(np.int8)
+    return q, _fp16_bits(s)
+
+
+def dequant_int8(q, s_bits):
+    from .rounding import fp16_value
+    s = fp16_value(s_bits)
+    return np.asarray(q, dtype=np.float64) * s[:, None]
+
+
+# --------------------------------------------------------------------- int4
+def quantize_int4(W, g):
+    """W float32 [N, K], group size g | K -> (q uint8 [N, K] in 0..15,
+    scale bits uint16 [N, K/g] bf16, zero bits uint16 [N, K/g] bf16).
+
+    Pinned by: |W - (q s + z)| <= s/2 per element, z <= min, z + 15 s >= max,
+    hand-computed groups (tests/golden), constant groups.
+    """
+    W = np.asarray(W, dtype=np.float32).astype(np.float64)
+    _check_finite(W)
+    N, K = W.shape
+    if g <= 0 or K % g:
+        raise ValueError("K must be a multiple of the group size")
+    Wg = W.reshape(N, K // g, g)
+    mn = Wg.min(axis=2)
+    mx = Wg.max(axis=2)
+    z = bf16_down(mn)
+    s = bf16_up((mx - z) / INT4_QMAX)
+    if np.any(np.isinf(s)) or np.any(np.isinf(z)):
+        raise ValueError("bf16 scale/zero overflow")
+    safe = np.where(s == 0, 1.0, s)
+    q = np.clip(np.rint((Wg - z[..., None]) / safe[..., None]), 0, INT4_QMAX)
+    q = np.where(s[..., None] == 0, 0, q).astype(np.uint8).reshape(N, K)
+    return q, _bf16_bits(s), _bf16_bits(z)
+
+
+def dequant_int4(q, s_bits, z_bits, g):
+    from .rounding import bf16_value
+    q = np.asarray(q, dtype=np.float64)
+    N, K = q.shape
+    s = np.repeat(bf16_value(s_bits), g, axis=1)
+    z = np.repeat(bf16_value(z_bits), g, axis=1)
+    return q * s + z
+
+
+# --------------------------------------------------------------------- helpers
+def _check_finite(W):
+    if not np.all(np.isfinite(W)):
+        raise ValueError("non-finite weight")
+
+
+def _fp16_bits(v):
+    from .rounding import fp16_bits
+    return fp16_bits(v)
+
+
+def _bf16_bits(v):
+    from .rounding import bf16_bits
+    return bf16_bits(v)

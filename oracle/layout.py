@@ -1,0 +1,99 @@
+"""Unpackers for the packed weight byte layouts, written from the layout definition.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).  These read a packed host
+buffer (bytes / uint8 array) bit by bit, following the layout as specified, and
+return the codes.  They are deliberately plain: Python integers and explicit
+bit positions, no shared tables with the library.
+
+Layout definition (the library's packers must produce exactly this):
+
+* int8:  byte n*K + k  =  q[n, k] + 128  (offset binary).
+* int4:  byte n*K/2 + k//2 holds q[n, k] in bits 0..3 if k is even, 4..7 if odd.
+* FP6 (2+4 split of each code c; sign = bit 5, e2 = bit 4, low piece = c & 0xF;
+  the split into a 2-bit and a 4-bit piece follows the FP6-LLM / TC-FPx
+  article, m.zhengruan.com news 124379, section "重新设计内核方案"):
+    - bytes [0, N*K/4): 2-bit plane; bytes [N*K/4, 3*N*K/4): 4-bit plane.
+    - 4-bit plane, little-endian 32-bit word t of row n at plane byte
+      n*K/2 + 4t, holds k = 8t + i, i = j + 4h (j in 0..3, h in 0..1); bit b of
+      the piece sits at word bit (5 + 16h - 4j + b) mod 32.
+    - 2-bit plane, little-endian 32-bit word u of row n at plane byte
+      n*K/4 + 4u, holds k = 16u + i, i = 8c + j + 4h; with
+      T = (0, 1, 4, 5, 8, 9, 12, 13)[4c + j] the sign bit sits at word bit
+      (15 + 16h - T) mod 32 and e2 at (9 + 16h - T) mod 32.
+* bf16: the plain row-major bf16 matrix (no packing).
+
+Pinned by hand-built byte examples in ``tests/golden/`` and by the
+pack -> unpack identity on one-hot, random, all-zero and all-max codes against
+the library's packers (tests/test_host_lib.py).
+"""
+
+import numpy as np
+
+_T = (0, 1, 4, 5, 8, 9, 12, 13)
+
+
+def _u8(buf):
+    return np.frombuffer(bytes(buf), dtype=np.uint8) if not isinstance(buf, np.ndarray) else buf.view(np.uint8).reshape(-1)
+
+
+def unpack_int8(packed, N, K):
+    """Packed int8 bytes -> q int8 [N, K]."""
+    b = _u8(packed)
+    assert b.size == N * K
+    return (b.astype(np.int16) - 128).astype(np.int8).reshape(N, K)
+
+
+def unpack_int4(packed, N, K):
+    """Packed int4 bytes -> q uint8 [N, K] (codes 0..15)."""
+    b = _u8(packed)
+    assert b.size == N * K // 2
+    q = np.empty((N, K), dtype=np.uint8)
+    for n in range(N):
+        row = b[n * K // 2:(n + 1) * K // 2]
+        for k in range(K):
+            byte = int(row[k // 2])
+            q[n, k] = (byte >> (4 * (k % 2))) & 0xF
+    return q
+
+
+def _word(plane, byte_off):
+    return int(plane[byte_off]) | (int(plane[byte_off + 1]) << 8) | (int(plane[byte_off + 2]) << 16) | (int(plane[byte_off + 3]) << 24)
+
+
+def _bit(word, pos):
+    return (word >> (pos % 32)) & 1
+
+
+def unpack_fp6(packed, N, K):
+    """Packed FP6 bytes -> codes uint8 [N, K] (0..63)."""
+    b = _u8(packed)
+    assert b.size == 3 * N * K // 4
+    p2 = b[:N * K // 4]
+    p4 = b[N * K // 4:]
+    codes = np.empty((N, K), dtype=np.uint8)
+    for n in range(N):
+        for k in range(K):
+            # 4-bit piece
+            t, i = divmod(k, 8)
+            j, h = i % 4, i // 4
+            w4 = _word(p4, n * K // 2 + 4 * t)
+            four = 0
+            for bb in range(4):
+                four |= _bit(w4, 5 + 16 * h - 4 * j + bb) << bb
+            # 2-bit piece
+            u, i16 = divmod(k, 16)
+            c, rest = divmod(i16, 8)
+            j2, h2 = rest % 4, rest // 4
+            T = _T[4 * c + j2]
+            w2 = _word(p2, n * K // 4 + 4 * u)
+            sign = _bit(w2, 15 + 16 * h2 - T)
+            e2 = _bit(w2, 9 + 16 * h2 - T)
+            codes[n, k] = (sign << 5) | (e2 << 4) | four
+    return codes
+
+
+def unpack_bf16(packed, N, K):
+    """Packed bf16 bytes -> uint16 bit patterns [N, K]."""
+    b = _u8(packed)
+    assert b.size == 2 * N * K
+    return b.view(np.uint16).reshape(N, K).copy()

@@ -1,0 +1,58 @@
+"""The decode linear y = x . deq(W)^T in float64, and its bf16 rounding.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
+
+The method (FP6-LLM / TC-FPx article, m.zhengruan.com news 124379, section
+"重新设计内核方案": dequantize the weights, then run an ordinary 16-bit matrix
+multiply; gpt-fast write-up, m.greenbasetech.com article 46368139_1106049486:
+weight-only quantization leaves the layer's result unchanged apart from the
+weights' rounding) reaches exactly - up to rounding order - the plain product of
+the bf16 activations with the dequantized weights.  So the oracle is that
+definition: ``y_ref = x . deq(W)^T`` in float64, and the bf16 output the kernel
+is held to is ``RNE_bf16(y_ref)``.
+
+``deq`` is one of ``oracle.formats.dequant_*``; x is given as bf16 bit patterns.
+
+Pinned by: a brute-force triple loop on tiny shapes (pure Python sums),
+the special case s = 1, z = 0 against numpy's matmul of the codes, and integer
+inputs whose exact result is known (tests/test_oracle.py).
+"""
+
+import numpy as np
+
+from .rounding import bf16_rne, bf16_value, bf16_bits
+from . import formats
+
+
+def deq_weights(fmt, codes, scales=None, zeros=None, g=None):
+    """Dequantized weights float64 [N, K] for fmt in {'int8','int4','fp6','bf16'}.
+
+    ``codes`` are the quantizer outputs (int8 q, int4 q, FP6 codes) or, for
+    'bf16', the uint16 bit patterns of W.
+    """
+    if fmt == "int8":
+        return formats.dequant_int8(codes, scales)
+    if fmt == "int4":
+        return formats.dequant_int4(codes, scales, zeros, g)
+    if fmt == "fp6":
+        return formats.dequant_fp6(codes, scales)
+    if fmt == "bf16":
+        return bf16_value(codes)
+    raise ValueError(fmt)
+
+
+def linear_ref(x_bits, Wd):
+    """float64 y [M, N] = x . Wd^T with x given as bf16 bit patterns [M, K]."""
+    x = bf16_value(x_bits)
+    return x @ np.asarray(Wd, dtype=np.float64).T
+
+
+def linear_ref_rows(x_bits, Wd_rows):
+    """Same as linear_ref for a subset of output channels (rows of W)."""
+    return linear_ref(x_bits, Wd_rows)
+
+
+def to_bf16(y):
+    """RNE bf16 rounding of float64 results: (values float64, bit patterns uint16)."""
+    v = bf16_rne(y)
+    return v, bf16_bits(v)

@@ -1,0 +1,267 @@
+"""Pins of the CPU oracle against what the formats and the mathematics fix.
+
+None of these compares the oracle with itself: each check uses a library
+routine (numpy / torch casts, numpy matmul), a hand-listed table or hand-worked
+example (tests/golden), a closed-form bound, or brute force.
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import formats, layout, linear, rounding
+import workloads
+
+
+# ------------------------------------------------------------------ helpers
+def _golden_lines(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def _parse_f32(tok):
+    if "p" in tok:
+        mant, exp = tok.split("p")
+        return float(np.float32(int(mant) * 2.0 ** int(exp)))
+    return float(np.float32(float(tok)))
+
+
+# ------------------------------------------------------------------ rounding
+def test_fp16_rne_matches_numpy_cast():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.integers(-9, 6, 20000),
+        # exact ties between two fp16 values (normal and subnormal)
+        (np.arange(1, 4000) + 0.5) * 2.0 ** -24,
+        (np.arange(1024, 3000) + 0.5) * 2.0 ** -10,
+        np.array([65504.0, 65519.99, 65520.0, 1e6, -1e6, 2.0 ** -25, 2.0 ** -26, 0.0, -0.0]),
+    ])
+    ours = rounding.fp16_rne(x)
+    with np.errstate(over="ignore"):
+        ref = x.astype(np.float16).astype(np.float64)
+    assert np.array_equal(ours, ref)
+    assert np.array_equal(np.signbit(ours), np.signbit(ref))
+
+
+def test_bf16_rne_matches_torch_cast():
+    rng = np.random.default_rng(2)
+    x32 = np.concatenate([
+        (rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000)).astype(np.float32),
+        # ties: bf16 value + half a bf16 spacing, exact in float32
+        ((np.arange(128, 256) + 0.5) * 2.0 ** -3).astype(np.float32),
+        np.array([1e-40, -3e-39, 3.3e38], dtype=np.float32),  # subnormals, near max
+    ])
+    ours = rounding.bf16_rne(x32.astype(np.float64))
+    ref = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_bf16_directed_rounding_brackets():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(5000) * 10.0 ** rng.integers(-5, 5, 5000)
+    lo = rounding.bf16_down(x)
+    hi = rounding.bf16_up(x)
+    assert np.all(lo <= x) and np.all(hi >= x)
+    # both are bf16 values (survive the library cast unchanged)
+    for v in (lo, hi):
+        assert np.array_equal(torch.tensor(v).to(torch.bfloat16).to(torch.float64).numpy(), v)
+    # and adjacent: no bf16 value strictly between them unless x itself is one
+    exact = lo == hi
+    bits_lo = rounding.bf16_bits(np.abs(lo[~exact]))
+    bits_hi = rounding.bf16_bits(np.abs(hi[~exact]))
+    assert np.all(np.abs(bits_hi.astype(np.int64) - bits_lo.astype(np.int64)) == 1)
+
+
+def test_bits_roundtrip():
+    v = np.array([0.0, 1.0, -2.5, 65504.0, 2.0 ** -24])
+    assert np.array_equal(rounding.fp16_value(rounding.fp16_bits(v)), v)
+    assert rounding.fp16_bits(np.array([1.0]))[0] == 0x3C00
+    assert rounding.bf16_bits(np.array([1.0]))[0] == 0x3F80
+    assert rounding.bf16_bits(np.array([-2.0]))[0] == 0xC000
+
+
+# ------------------------------------------------------------------ e3m2
+def test_e3m2_table_matches_hand_list(golden_dir):
+    rows = _golden_lines(golden_dir, "e3m2_magnitudes.txt")
+    table = {int(c): float(v) for c, v in rows}
+    assert sorted(table) == list(range(32))
+    got = formats.e3m2_value(np.arange(64))
+    for c in range(32):
+        assert got[c] == table[c]
+        assert got[c + 32] == -table[c]
+
+
+def test_e3m2_closed_form_properties():
+    v = formats.e3m2_value(np.arange(32))
+    assert v.max() == 28.0
+    assert v[v > 0].min() == 0.0625
+    assert np.all(np.diff(v) > 0)  # monotone in the code
+    assert formats.e3m2_value(32) == 0.0  # negative zero decodes to 0
+
+
+# ------------------------------------------------------------------ quantizers
+def test_int8_hand_example(golden_dir):
+    rows = {tuple(r[:2]): r[2:] for r in _golden_lines(golden_dir, "quant_examples.txt") if r[0] == "int8"}
+    W = np.array([[_parse_f32(t) for t in rows[("int8", "W")]]], dtype=np.float32)
+    q, s = formats.quantize_int8(W)
+    assert q.tolist()[0] == [int(t) for t in rows[("int8", "q")]]
+    assert int(s[0]) == int(rows[("int8", "s")][0], 16)
+
+
+def test_int4_hand_example(golden_dir):
+    rows = {tuple(r[:2]): r[2:] for r in _golden_lines(golden_dir, "quant_examples.txt") if r[0] == "int4"}
+    g = int(rows[("int4", "g")][0])
+    W = np.array([[_parse_f32(t) for t in rows[("int4", "W")]]], dtype=np.float32)
+    q, s, z = formats.quantize_int4(W, g)
+    assert q.tolist()[0] == [int(t) for t in rows[("int4", "q")]]
+    assert int(s[0, 0]) == int(rows[("int4", "s")][0], 16)
+    assert int(z[0, 0]) == int(rows[("int4", "z")][0], 16)
+
+
+def test_fp6_hand_example(golden_dir):
+    rows = {tuple(r[:2]): r[2:] for r in _golden_lines(golden_dir, "quant_examples.txt") if r[0] == "fp6"}
+    W = np.array([[_parse_f32(t) for t in rows[("fp6", "W")]]], dtype=np.float32)
+    c, s = formats.quantize_fp6(W)
+    assert c.tolist()[0] == [int(t) for t in rows[("fp6", "code")]]
+    assert int(s[0]) == int(rows[("fp6", "s")][0], 16)
+
+
+def _w(N, K, seed):
+    return workloads.weights(N, K, seed).numpy()
+
+
+def test_int8_roundtrip_bound():
+    W = _w(64, 512, 11)
+    q, sb = formats.quantize_int8(W)
+    s = rounding.fp16_value(sb)
+    err = np.abs(W.astype(np.float64) - formats.dequant_int8(q, sb))
+    assert np.all(err <= s[:, None] / 2 * (1 + 1e-12))
+    assert q.min() >= -127 and q.max() <= 127
+    # the largest-magnitude element of each row maps to +-127 (scale ~ amax/127)
+    assert np.all(np.abs(q).max(axis=1) >= 126)
+
+
+def test_int4_roundtrip_bound_and_bracket():
+    W = _w(32, 512, 12)
+    for g in (32, 64, 128):
+        q, sb, zb = formats.quantize_int4(W, g)
+        s = rounding.bf16_value(sb)
+        z = rounding.bf16_value(zb)
+        Wg = W.astype(np.float64).reshape(32, 512 // g, g)
+        assert np.all(z <= Wg.min(axis=2))
+        assert np.all(z + 15 * s >= Wg.max(axis=2) * (1 - 1e-12) - 1e-30)
+        err = np.abs(W - formats.dequant_int4(q, sb, zb, g))
+        assert np.all(err <= np.repeat(s, g, axis=1) / 2 * (1 + 1e-9))
+        assert q.max() <= 15
+
+
+def test_int4_constant_group():
+    W = np.full((2, 64), 0.375, dtype=np.float32)  # exactly a bf16 value
+    q, sb, zb = formats.quantize_int4(W, 32)
+    assert np.all(q == 0)
+    assert np.all(rounding.bf16_value(sb) == 0.0)
+    assert np.all(formats.dequant_int4(q, sb, zb, 32) == 0.375)
+
+
+def test_fp6_rounding_is_nearest():
+    W = _w(32, 512, 13)
+    c, sb = formats.quantize_fp6(W)
+    s = rounding.fp16_value(sb)
+    r = W.astype(np.float64) / s[:, None]
+    v = formats.e3m2_value(c)
+    grid = np.concatenate([-formats.e3m2_value(np.arange(31, 0, -1)), formats.e3m2_value(np.arange(32))])
+    # distance to the chosen value is the minimum distance to any grid point
+    dmin = np.min(np.abs(r[..., None] - grid), axis=-1)
+    assert np.all(np.abs(r - v) <= dmin + 1e-12)
+    assert np.all(np.abs(v) <= 28.0)
+
+
+def test_fp6_saturates_and_zero_rows():
+    W = np.zeros((2, 64), dtype=np.float32)
+    W[1, 0] = 1.0
+    W[1, 1] = -1.0
+    c, sb = formats.quantize_fp6(W)
+    assert np.all(c[0] == 0) and sb[0] == 0
+    assert c[1, 0] == 31 and c[1, 1] == 63  # +-28 at the row maximum
+
+
+def test_zero_rows_int8():
+    q, sb = formats.quantize_int8(np.zeros((3, 64), dtype=np.float32))
+    assert np.all(q == 0) and np.all(sb == 0)
+
+
+def test_quantizers_reject_nonfinite():
+    W = np.zeros((1, 64), dtype=np.float32)
+    W[0, 3] = np.inf
+    for f in (formats.quantize_int8, formats.quantize_fp6, lambda w: formats.quantize_int4(w, 32)):
+        with pytest.raises(ValueError):
+            f(W)
+
+
+# ------------------------------------------------------------------ layout
+def test_fp6_layout_hand_examples(golden_dir):
+    rows = _golden_lines(golden_dir, "fp6_layout_examples.txt")
+    pairs = [(rows[i], rows[i + 1]) for i in range(0, len(rows), 2)]
+    assert len(pairs) == 3
+    for codes_line, bytes_line in pairs:
+        assert codes_line[0] == "codes" and bytes_line[0] == "bytes"
+        codes = [int(t) for t in codes_line[1:]]
+        buf = bytes(int(t, 16) for t in bytes_line[1:])
+        got = layout.unpack_fp6(buf, 1, 16)
+        assert got.tolist()[0] == codes
+
+
+def test_int4_int8_layout_hand_examples():
+    # int4: k = 0 -> low nibble, k = 1 -> high nibble of byte 0
+    buf = bytes([0x21, 0x0F] + [0] * 30)
+    q = layout.unpack_int4(buf, 1, 64)
+    assert q[0, :4].tolist() == [1, 2, 15, 0]
+    # int8 offset binary: 0x80 -> 0, 0x00 -> -128 (never produced), 0xFF -> 127, 0x01 -> -127
+    q8 = layout.unpack_int8(bytes([0x80, 0xFF, 0x01] + [0x80] * 61), 1, 64)
+    assert q8[0, :3].tolist() == [0, 127, -127]
+
+
+# ------------------------------------------------------------------ linear
+def test_linear_brute_force_tiny():
+    rng = np.random.default_rng(5)
+    M, N, K = 3, 5, 64
+    x = workloads.activations(M, K, 7)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    Wd = rng.standard_normal((N, K))
+    y = linear.linear_ref(xb, Wd)
+    xv = rounding.bf16_value(xb)
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += float(xv[m, k]) * float(Wd[n, k])
+            assert abs(acc - y[m, n]) <= 1e-12 * (1 + abs(acc))
+
+
+def test_linear_identity_scales_is_matmul_of_codes():
+    rng = np.random.default_rng(6)
+    q = rng.integers(-127, 128, (16, 128)).astype(np.int8)
+    one = np.full(16, 0x3C00, dtype=np.uint16)  # fp16 1.0
+    x = workloads.activations(2, 128, 8)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    y = linear.linear_ref(xb, linear.deq_weights("int8", q, one))
+    ref = x.to(torch.float64).numpy() @ q.astype(np.float64).T
+    assert np.array_equal(y, ref)
+    # int4 with s = 1, z = 0
+    q4 = rng.integers(0, 16, (16, 128)).astype(np.uint8)
+    s1 = np.full((16, 4), 0x3F80, dtype=np.uint16)
+    z0 = np.zeros((16, 4), dtype=np.uint16)
+    y4 = linear.linear_ref(xb, linear.deq_weights("int4", q4, s1, z0, 32))
+    assert np.array_equal(y4, x.to(torch.float64).numpy() @ q4.astype(np.float64).T)
+
+
+def test_linear_integer_exact():
+    # integer x and integer weights: the exact result is an integer sum
+    x = workloads.integer_activations(2, 128, 9)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    W = np.arange(-64, 64, dtype=np.float64)[None, :].repeat(3, axis=0)
+    y = linear.linear_ref(xb, W)
+    xi = x.to(torch.int64).numpy()
+    assert np.array_equal(y, (xi @ np.arange(-64, 64)[:, None].repeat(3, axis=1)).astype(np.float64))
