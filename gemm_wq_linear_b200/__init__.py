@@ -1,0 +1,243 @@
+"""Thin Python binding of libwq (ctypes): the same entry points as include/wq.h.
+
+Only argument marshalling happens here: torch tensors are turned into raw
+pointers, sizes and the current CUDA stream.  Every step of the computation runs
+in libwq's code (host packers / quantizers, sm_100a kernels).  There is no
+fallback: if libwq.so is missing or fails to load, importing this package
+raises.
+
+Host-side entry points take CPU tensors and return CPU tensors; compute entry
+points take CUDA tensors (16-byte aligned, contiguous) and run asynchronously
+on ``torch.cuda.current_stream()`` unless a stream is given.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwq.so")
+
+WQ_INT8, WQ_INT4, WQ_FP6_E3M2, WQ_BF16 = 0, 1, 2, 3
+FMT = {"int8": WQ_INT8, "int4": WQ_INT4, "fp6": WQ_FP6_E3M2, "bf16": WQ_BF16}
+WQ_LAUNCH_PDL = 0x1
+STATUS = {0: "WQ_OK", 1: "WQ_ERR_NULL", 2: "WQ_ERR_SHAPE", 3: "WQ_ERR_FMT", 4: "WQ_ERR_GROUP",
+          5: "WQ_ERR_ALIGN", 6: "WQ_ERR_CUDA", 7: "WQ_ERR_RANGE", 8: "WQ_ERR_TIMEOUT"}
+
+EXPORTS = (
+    "wq_packed_size", "wq_scales_size", "wq_quantize_int8", "wq_quantize_int4", "wq_quantize_fp6",
+    "wq_pack_int8", "wq_pack_int4", "wq_prepack_fp6", "wq_linear", "wq_linear_ex", "wq_unpack_debug",
+    "wq_sync_status", "wq_last_error", "wq_version",
+)
+
+
+class WQError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m gemm_wq_linear_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint
+    sig = {
+        "wq_packed_size": (ctypes.c_size_t, [i32, i64, i64]),
+        "wq_scales_size": (ctypes.c_size_t, [i32, i64, i64, i32]),
+        "wq_quantize_int8": (i32, [vp, i64, i64, vp, vp]),
+        "wq_quantize_int4": (i32, [vp, i64, i64, i32, vp, vp, vp]),
+        "wq_quantize_fp6": (i32, [vp, i64, i64, vp, vp]),
+        "wq_pack_int8": (i32, [vp, i64, i64, vp]),
+        "wq_pack_int4": (i32, [vp, i64, i64, vp]),
+        "wq_prepack_fp6": (i32, [vp, i64, i64, vp]),
+        "wq_linear": (i32, [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp]),
+        "wq_linear_ex": (i32, [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, u32]),
+        "wq_unpack_debug": (i32, [vp, i32, i64, i64, vp, vp]),
+        "wq_sync_status": (i32, [vp]),
+        "wq_last_error": (ctypes.c_char_p, []),
+        "wq_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status):
+    if status != 0:
+        raise WQError(status, lib.wq_last_error().decode())
+
+
+def _fmt(fmt):
+    return FMT[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _host(t, dtype):
+    if t.device.type != "cpu" or t.dtype != dtype or not t.is_contiguous():
+        raise TypeError(f"expected a contiguous CPU {dtype} tensor")
+    return t
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------------ sizes
+def wq_packed_size(fmt, N, K):
+    return int(lib.wq_packed_size(_fmt(fmt), N, K))
+
+
+def wq_scales_size(fmt, N, K, groupsize=0):
+    return int(lib.wq_scales_size(_fmt(fmt), N, K, groupsize))
+
+
+def wq_version():
+    return lib.wq_version().decode()
+
+
+# ------------------------------------------------------------------ quantizers (host)
+def wq_quantize_int8(W):
+    """W float32 [N, K] CPU -> (q int8 [N, K], s int16 [N] holding fp16 bits)."""
+    _host(W, torch.float32)
+    N, K = W.shape
+    q = torch.empty(N, K, dtype=torch.int8)
+    s = torch.empty(N, dtype=torch.int16)
+    _check(lib.wq_quantize_int8(_ptr(W), N, K, _ptr(q), _ptr(s)))
+    return q, s
+
+
+def wq_quantize_int4(W, groupsize):
+    """W float32 [N, K] CPU -> (q uint8 [N, K], s int16 [N, K/g] bf16 bits, z int16 [N, K/g] bf16 bits)."""
+    _host(W, torch.float32)
+    N, K = W.shape
+    G = K // groupsize if groupsize > 0 else 0
+    q = torch.empty(N, K, dtype=torch.uint8)
+    s = torch.empty(N, max(G, 0), dtype=torch.int16)
+    z = torch.empty(N, max(G, 0), dtype=torch.int16)
+    _check(lib.wq_quantize_int4(_ptr(W), N, K, groupsize, _ptr(q), _ptr(s), _ptr(z)))
+    return q, s, z
+
+
+def wq_quantize_fp6(W):
+    """W float32 [N, K] CPU -> (codes uint8 [N, K], s int16 [N] holding fp16 bits)."""
+    _host(W, torch.float32)
+    N, K = W.shape
+    c = torch.empty(N, K, dtype=torch.uint8)
+    s = torch.empty(N, dtype=torch.int16)
+    _check(lib.wq_quantize_fp6(_ptr(W), N, K, _ptr(c), _ptr(s)))
+    return c, s
+
+
+# ------------------------------------------------------------------ packers (host)
+def wq_pack_int8(q):
+    _host(q, torch.int8)
+    N, K = q.shape
+    out = torch.empty(wq_packed_size("int8", N, K), dtype=torch.uint8)
+    _check(lib.wq_pack_int8(_ptr(q), N, K, _ptr(out)))
+    return out
+
+
+def wq_pack_int4(q):
+    _host(q, torch.uint8)
+    N, K = q.shape
+    out = torch.empty(wq_packed_size("int4", N, K), dtype=torch.uint8)
+    _check(lib.wq_pack_int4(_ptr(q), N, K, _ptr(out)))
+    return out
+
+
+def wq_prepack_fp6(codes):
+    _host(codes, torch.uint8)
+    N, K = codes.shape
+    out = torch.empty(wq_packed_size("fp6", N, K), dtype=torch.uint8)
+    _check(lib.wq_prepack_fp6(_ptr(codes), N, K, _ptr(out)))
+    return out
+
+
+# ------------------------------------------------------------------ compute (device)
+def wq_linear(x, packed, scales, zeros, y, M, N, K, fmt, groupsize=0, stream=None):
+    _check(lib.wq_linear(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(y), M, N, K, _fmt(fmt),
+                         groupsize, _stream(stream)))
+
+
+def wq_linear_ex(x, packed, scales, zeros, y, M, N, K, fmt, groupsize=0, stream=None, flags=0):
+    _check(lib.wq_linear_ex(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(y), M, N, K, _fmt(fmt),
+                            groupsize, _stream(stream), flags))
+
+
+def wq_unpack_debug(packed, fmt, N, K, out, stream=None):
+    _check(lib.wq_unpack_debug(_ptr(packed), _fmt(fmt), N, K, _ptr(out), _stream(stream)))
+
+
+def wq_sync_status(stream=None):
+    _check(lib.wq_sync_status(_stream(stream)))
+
+
+# ------------------------------------------------------------------ convenience
+class PackedWeight:
+    """Device-resident packed weight of one linear layer (buffers owned by torch)."""
+
+    def __init__(self, fmt, N, K, packed, scales=None, zeros=None, groupsize=0):
+        self.fmt, self.N, self.K, self.groupsize = _fmt(fmt), N, K, groupsize
+        self.packed, self.scales, self.zeros = packed, scales, zeros
+
+    @classmethod
+    def from_codes(cls, fmt, codes, scales=None, zeros=None, groupsize=0, device="cuda"):
+        """Pack host codes (quantizer outputs, or bf16 bits as int16 for 'bf16') and upload."""
+        f = _fmt(fmt)
+        N, K = codes.shape
+        if f == WQ_INT8:
+            p = wq_pack_int8(codes)
+        elif f == WQ_INT4:
+            p = wq_pack_int4(codes)
+        elif f == WQ_FP6_E3M2:
+            p = wq_prepack_fp6(codes)
+        else:
+            p = codes.contiguous().view(torch.uint8).reshape(-1)
+        dev = lambda t: None if t is None else t.contiguous().to(device)
+        return cls(f, N, K, dev(p), dev(scales), dev(zeros), groupsize)
+
+    @classmethod
+    def quantize(cls, W, fmt, groupsize=0, device="cuda"):
+        """Quantize a float32 CPU weight [N, K] with libwq's quantizer, pack and upload."""
+        f = _fmt(fmt)
+        if f == WQ_INT8:
+            q, s = wq_quantize_int8(W)
+            return cls.from_codes(f, q, s, device=device)
+        if f == WQ_INT4:
+            q, s, z = wq_quantize_int4(W, groupsize)
+            return cls.from_codes(f, q, s, z, groupsize, device=device)
+        if f == WQ_FP6_E3M2:
+            c, s = wq_quantize_fp6(W)
+            return cls.from_codes(f, c, s, device=device)
+        return cls.from_codes(f, W.to(torch.bfloat16).view(torch.int16), device=device)
+
+    def nbytes(self):
+        n = self.packed.numel()
+        for t in (self.scales, self.zeros):
+            if t is not None:
+                n += t.numel() * t.element_size()
+        return n
+
+
+def linear(x, pw, out=None, stream=None, flags=0):
+    """y = x . deq(W)^T for a bf16 CUDA tensor x [M, K] and a PackedWeight."""
+    M, K = x.shape
+    if K != pw.K:
+        raise ValueError("K mismatch")
+    y = out if out is not None else torch.empty(M, pw.N, dtype=torch.bfloat16, device=x.device)
+    wq_linear_ex(x, pw.packed, pw.scales, pw.zeros, y, M, pw.N, K, pw.fmt, pw.groupsize, stream, flags)
+    return y

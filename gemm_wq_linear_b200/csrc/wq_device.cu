@@ -1,0 +1,196 @@
+// Device-side entry points of the wq C ABI: argument checks, dispatch, the
+// decode-only test kernel and the status query.
+#include "wq_internal.h"
+#include "wq_kernels.cuh"
+#include "decode.cuh"
+
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+namespace wq {
+
+// Number of SMs of each device, cached (cudaDeviceGetAttribute is cheap but
+// this keeps wq_linear free of any query on the hot path).
+static int sm_count_of_current_device() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Largest K: bounds the per-CTA shared memory of the GEMV partial sums.
+static const int kMaxK = 262144;
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------ unpack debug
+// One thread per 32 consecutive weights of a row: the same decoders as the
+// compute kernels, followed by the exact removal of the decode offsets, written
+// back in k order.
+__global__ void unpack_debug_kernel(const uint8_t* __restrict__ packed, int fmt, int N, int K,
+                                    uint16_t* __restrict__ out) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long per_row = K / 32;
+  if (tid >= (long long)N * per_row) return;
+  const int n = int(tid / per_row);
+  const int k0 = int(tid - (long long)n * per_row) * 32;
+  float v[32];
+  if (fmt == WQ_INT4) {
+    const uint4 w = *reinterpret_cast<const uint4*>(packed + size_t(n) * (K / 2) + k0 / 2);
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    for (int q = 0; q < 4; ++q) {
+      uint32_t p[4];
+      decode_int4_word(words[q], p);
+      for (int r = 0; r < 4; ++r) {
+        v[8 * q + r] = bf16_lo_f(p[r]) - 128.f;
+        v[8 * q + r + 4] = bf16_hi_f(p[r]) - 128.f;
+      }
+    }
+  } else if (fmt == WQ_FP6_E3M2) {
+    const uint8_t* p2 = packed;
+    const uint8_t* p4 = packed + size_t(N) * (K / 4);
+    const uint4 w4 = *reinterpret_cast<const uint4*>(p4 + size_t(n) * (K / 2) + k0 / 2);
+    const uint2 w2 = *reinterpret_cast<const uint2*>(p2 + size_t(n) * (K / 4) + k0 / 4);
+    const uint32_t a4[4] = {w4.x, w4.y, w4.z, w4.w};
+    const uint32_t a2[2] = {w2.x, w2.y};
+    const uint32_t one = 0x3F803F80u;  // bf16 (1, 1)
+    for (int u = 0; u < 2; ++u) {
+      uint32_t p[8];
+      decode_fp6_words(a2[u], a4[2 * u], a4[2 * u + 1], p);
+      for (int c = 0; c < 2; ++c)
+        for (int j = 0; j < 4; ++j) {
+          // the compute path multiplies the scaled code with bf16 activations
+          // in fp32 and rescales by 2^124 at the end; mirror that with x = 1
+          float lo = 0.f, hi = 0.f;
+          fma_bf16_lo(lo, p[4 * c + j], one);
+          fma_bf16_hi(hi, p[4 * c + j], one);
+          v[16 * u + 8 * c + j] = lo * 0x1p124f;
+          v[16 * u + 8 * c + j + 4] = hi * 0x1p124f;
+        }
+    }
+  } else if (fmt == WQ_INT8) {
+    const uint8_t* base = packed + size_t(n) * K + k0;
+    for (int q = 0; q < 4; ++q) {
+      const uint2 w = *reinterpret_cast<const uint2*>(base + 8 * q);
+      decode_int8_word(w.x, v + 8 * q);
+      decode_int8_word(w.y, v + 8 * q + 4);
+    }
+  } else {
+    const uint16_t* base = reinterpret_cast<const uint16_t*>(packed) + size_t(n) * K + k0;
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(uint32_t(base[i]) << 16);
+  }
+  uint4* o = reinterpret_cast<uint4*>(out + size_t(n) * K + k0);
+  for (int q = 0; q < 4; ++q) {
+    uint4 r;
+    r.x = pack_bf16x2_rn(v[8 * q + 0], v[8 * q + 1]);
+    r.y = pack_bf16x2_rn(v[8 * q + 2], v[8 * q + 3]);
+    r.z = pack_bf16x2_rn(v[8 * q + 4], v[8 * q + 5]);
+    r.w = pack_bf16x2_rn(v[8 * q + 6], v[8 * q + 7]);
+    o[q] = r;
+  }
+}
+
+cudaError_t launch_unpack_debug(const void* packed, int fmt, int N, int K, uint16_t* out, cudaStream_t s) {
+  const long long threads = (long long)N * (K / 32);
+  const int block = 256;
+  const long long grid = (threads + block - 1) / block;
+  unpack_debug_kernel<<<unsigned(grid), block, 0, s>>>(static_cast<const uint8_t*>(packed), fmt, N, K, out);
+  return cudaGetLastError();
+}
+
+static wq_status check_shape(const char* fn, int64_t M, int64_t N, int64_t K, int fmt, int groupsize) {
+  if (fmt < WQ_INT8 || fmt > WQ_BF16) return set_error(WQ_ERR_FMT, "%s: unknown format %d", fn, fmt);
+  if (M < 0 || M > 32) return set_error(WQ_ERR_SHAPE, "%s: M = %lld outside [0, 32]", fn, (long long)M);
+  if (N < 0 || K < 0 || K % 64)
+    return set_error(WQ_ERR_SHAPE, "%s: need N >= 0, K >= 0, K %% 64 == 0 (N = %lld, K = %lld)", fn, (long long)N,
+                     (long long)K);
+  if (N > (1 << 30) || K > kMaxK || N * K > (int64_t(1) << 31) - 1)
+    return set_error(WQ_ERR_SHAPE, "%s: need K <= %d and N * K < 2^31 (N = %lld, K = %lld)", fn, kMaxK,
+                     (long long)N, (long long)K);
+  if (fmt == WQ_INT4 && (!valid_group(groupsize) || K % groupsize))
+    return set_error(WQ_ERR_GROUP, "%s: int4 group size %d must be 32, 64 or 128 and divide K = %lld", fn, groupsize,
+                     (long long)K);
+  return WQ_OK;
+}
+
+}  // namespace wq
+
+using namespace wq;
+
+extern "C" {
+
+wq_status wq_linear_ex(const void* x, const void* packed, const void* scales, const void* zeros, void* y,
+                       int64_t M, int64_t N, int64_t K, int fmt, int groupsize, void* cuda_stream,
+                       unsigned flags) {
+  static const char* fn = "wq_linear";
+  wq_status st = check_shape(fn, M, N, K, fmt, groupsize);
+  if (st != WQ_OK) return st;
+  if (flags & ~WQ_LAUNCH_PDL) return set_error(WQ_ERR_SHAPE, "%s: unknown flags 0x%x", fn, flags);
+  if (M == 0 || N == 0) return ok();
+  if (!x || !packed || !y) return set_error(WQ_ERR_NULL, "%s: x, packed and y must be non-null", fn);
+  if (fmt != WQ_BF16 && !scales) return set_error(WQ_ERR_NULL, "%s: scales must be non-null", fn);
+  if (fmt == WQ_BF16 && scales) return set_error(WQ_ERR_NULL, "%s: scales must be NULL for bf16 weights", fn);
+  if ((fmt == WQ_INT4) != (zeros != nullptr))
+    return set_error(WQ_ERR_NULL, "%s: zeros must be non-null for int4 and NULL otherwise", fn);
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(y) || (scales && !aligned16(scales)) ||
+      (zeros && !aligned16(zeros)))
+    return set_error(WQ_ERR_ALIGN, "%s: device pointers must be 16-byte aligned", fn);
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (K == 0) {
+    cudaError_t e = cudaMemsetAsync(y, 0, size_t(M) * size_t(N) * 2, stream);
+    if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+    return ok();
+  }
+  const int sms = sm_count_of_current_device();
+  GemvParams p{};
+  p.packed = packed;
+  p.scales = static_cast<const uint16_t*>(scales);
+  p.zeros = static_cast<const uint16_t*>(zeros);
+  p.N = int(N);
+  p.K = int(K);
+  p.groupsize = groupsize;
+  p.fmt = fmt;
+  p.pdl = (flags & WQ_LAUNCH_PDL) ? 1 : 0;
+  for (int64_t m0 = 0; m0 < M; m0 += 4) {
+    p.M = int(M - m0 < 4 ? M - m0 : 4);
+    p.x = static_cast<const uint16_t*>(x) + m0 * K;
+    p.y = static_cast<uint16_t*>(y) + m0 * N;
+    cudaError_t e = launch_gemv(p, stream, sms);
+    if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  }
+  return ok();
+}
+
+wq_status wq_linear(const void* x, const void* packed, const void* scales, const void* zeros, void* y, int64_t M,
+                    int64_t N, int64_t K, int fmt, int groupsize, void* cuda_stream) {
+  return wq_linear_ex(x, packed, scales, zeros, y, M, N, K, fmt, groupsize, cuda_stream, 0u);
+}
+
+wq_status wq_unpack_debug(const void* packed, int fmt, int64_t N, int64_t K, void* out_bf16, void* cuda_stream) {
+  static const char* fn = "wq_unpack_debug";
+  wq_status st = check_shape(fn, 1, N, K, fmt, fmt == WQ_INT4 ? 32 : 0);
+  if (st != WQ_OK && !(fmt == WQ_INT4 && st == WQ_ERR_GROUP)) return st;
+  if (N == 0 || K == 0) return ok();
+  if (!packed || !out_bf16) return set_error(WQ_ERR_NULL, "%s: null pointer", fn);
+  if (!aligned16(packed) || !aligned16(out_bf16)) return set_error(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned", fn);
+  cudaError_t e = launch_unpack_debug(packed, fmt, int(N), int(K), static_cast<uint16_t*>(out_bf16),
+                                      static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  return ok();
+}
+
+wq_status wq_sync_status(void* cuda_stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "wq_sync_status: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,309 @@
+// Host side of the wq C ABI: error state, buffer sizes, offline quantizers and
+// packers.  Everything here runs on the CPU and touches only host memory.
+//
+// Quantizers implement the format definitions of include/wq.h with integer
+// rounding on IEEE-754 bit patterns (no libm rounding helpers except nearbyint
+// in the default round-to-nearest-even mode).
+#include "wq_internal.h"
+
+#include <cfenv>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+namespace wq {
+
+static thread_local std::string g_last_error;
+
+wq_status set_error(wq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+wq_status ok() {
+  g_last_error.clear();
+  return WQ_OK;
+}
+
+const char* last_error() { return g_last_error.c_str(); }
+
+// ------------------------------------------------------------------ rounding
+// Round a positive finite double onto a binary format with `frac` explicit
+// fraction bits and minimum normal exponent `emin`, using the integer
+// significand of the double.  mode: 0 = nearest-even, +1 = up, -1 = down
+// (applied to the magnitude; callers map signed directed rounding onto it).
+// Returns the rounded magnitude as a double (may be +inf-free: caller checks).
+static double round_mag(double a, int frac, int emin, int mode) {
+  if (a == 0.0) return 0.0;
+  uint64_t bits;
+  std::memcpy(&bits, &a, 8);
+  int bexp = int((bits >> 52) & 0x7FF);
+  uint64_t sig = bits & ((uint64_t(1) << 52) - 1);
+  int E;
+  if (bexp == 0) {  // double subnormal: value = sig * 2^-1074
+    E = -1074 + 52;
+    while (!(sig & (uint64_t(1) << 52))) {
+      sig <<= 1;
+      --E;
+    }
+  } else {
+    sig |= uint64_t(1) << 52;
+    E = bexp - 1023;
+  }
+  // value = sig * 2^(E - 52).  Target grid spacing is 2^(max(E, emin) - frac).
+  int Eg = E < emin ? emin : E;
+  int shift = (Eg - frac) - (E - 52);  // number of low bits of sig below the grid
+  if (shift <= 0) return a;  // already on the grid (cannot happen for frac < 52)
+  if (shift >= 64) {         // far below half a grid step
+    return mode > 0 ? std::ldexp(1.0, Eg - frac) : 0.0;
+  }
+  uint64_t kept = sig >> shift;
+  const uint64_t rem = sig & ((uint64_t(1) << shift) - 1);
+  const uint64_t half = uint64_t(1) << (shift - 1);
+  if (mode == 0) {
+    if (rem > half || (rem == half && (kept & 1))) ++kept;
+  } else if (mode > 0) {
+    if (rem) ++kept;
+  }
+  return std::ldexp(double(kept), Eg - frac);
+}
+
+static uint16_t fp16_bits_of(double v) {  // v exactly representable in fp16, finite
+  uint16_t s = std::signbit(v) ? 0x8000 : 0;
+  double a = std::fabs(v);
+  if (a == 0.0) return s;
+  int e;
+  double f = std::frexp(a, &e);  // a = f * 2^e, f in [0.5, 1)
+  int E = e - 1;                 // a = (2f) * 2^E
+  if (E < -14) {                 // subnormal: a = m * 2^-24
+    return uint16_t(s | uint16_t(std::ldexp(a, 24)));
+  }
+  uint16_t m = uint16_t(std::ldexp(2.0 * f - 1.0, 10));
+  return uint16_t(s | uint16_t((E + 15) << 10) | m);
+}
+
+static uint16_t bf16_bits_of(double v) {  // v exactly representable in bf16, finite
+  float f = float(v);
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return uint16_t(u >> 16);
+}
+
+static const double kFp16Max = 65504.0;
+static const double kBf16Max = 3.3895313892515355e38;  // (2 - 2^-7) * 2^127
+
+// fp16 round-to-nearest-even of a non-negative double; returns +inf on overflow.
+static double fp16_rne_pos(double a) {
+  double r = round_mag(a, 10, -14, 0);
+  return r > kFp16Max ? INFINITY : r;
+}
+
+// bf16 directed rounding of a signed double (toward -inf / +inf).
+static double bf16_floor(double x) {
+  double r = x >= 0 ? round_mag(x, 7, -126, -1) : -round_mag(-x, 7, -126, +1);
+  return r;
+}
+static double bf16_ceil(double x) {
+  double r = x >= 0 ? round_mag(x, 7, -126, +1) : -round_mag(-x, 7, -126, -1);
+  return r;
+}
+
+static bool all_finite(const float* W, int64_t n) {
+  for (int64_t i = 0; i < n; ++i)
+    if (!std::isfinite(W[i])) return false;
+  return true;
+}
+
+}  // namespace wq
+
+using namespace wq;
+
+extern "C" {
+
+const char* wq_last_error(void) { return last_error(); }
+
+const char* wq_version(void) { return "wq 0.1 sm_100a"; }
+
+size_t wq_packed_size(int fmt, int64_t N, int64_t K) {
+  if (N < 0 || K < 0) return 0;
+  const size_t nk = size_t(N) * size_t(K);
+  switch (fmt) {
+    case WQ_INT8: return nk;
+    case WQ_INT4: return nk / 2;
+    case WQ_FP6_E3M2: return nk / 4 * 3;
+    case WQ_BF16: return nk * 2;
+    default: return 0;
+  }
+}
+
+size_t wq_scales_size(int fmt, int64_t N, int64_t K, int groupsize) {
+  if (N < 0 || K < 0) return 0;
+  switch (fmt) {
+    case WQ_INT8:
+    case WQ_FP6_E3M2: return size_t(N) * 2;
+    case WQ_INT4:
+      if (!valid_group(groupsize) || K % groupsize) return 0;
+      return size_t(N) * size_t(K / groupsize) * 2;
+    default: return 0;
+  }
+}
+
+wq_status wq_quantize_int8(const float* W, int64_t N, int64_t K, int8_t* q, uint16_t* s_fp16) {
+  if (!W || !q || !s_fp16) return set_error(WQ_ERR_NULL, "wq_quantize_int8: null pointer");
+  if (N < 0 || K < 0) return set_error(WQ_ERR_SHAPE, "wq_quantize_int8: negative shape");
+  if (!all_finite(W, N * K)) return set_error(WQ_ERR_RANGE, "wq_quantize_int8: non-finite weight");
+  std::fesetround(FE_TONEAREST);
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    double amax = 0.0;
+    for (int64_t k = 0; k < K; ++k) amax = std::fmax(amax, std::fabs(double(w[k])));
+    double s = fp16_rne_pos(amax / 127.0);
+    if (std::isinf(s)) return set_error(WQ_ERR_RANGE, "wq_quantize_int8: fp16 scale overflow in row %lld", (long long)n);
+    s_fp16[n] = fp16_bits_of(s);
+    for (int64_t k = 0; k < K; ++k) {
+      double v = s == 0.0 ? 0.0 : std::nearbyint(double(w[k]) / s);
+      v = v > 127.0 ? 127.0 : (v < -127.0 ? -127.0 : v);
+      q[n * K + k] = int8_t(v);
+    }
+  }
+  return ok();
+}
+
+wq_status wq_quantize_int4(const float* W, int64_t N, int64_t K, int groupsize, uint8_t* q,
+                           uint16_t* s_bf16, uint16_t* z_bf16) {
+  if (!W || !q || !s_bf16 || !z_bf16) return set_error(WQ_ERR_NULL, "wq_quantize_int4: null pointer");
+  if (N < 0 || K < 0) return set_error(WQ_ERR_SHAPE, "wq_quantize_int4: negative shape");
+  if (groupsize <= 0 || K % groupsize)
+    return set_error(WQ_ERR_GROUP, "wq_quantize_int4: group size %d does not divide K = %lld", groupsize, (long long)K);
+  if (!all_finite(W, N * K)) return set_error(WQ_ERR_RANGE, "wq_quantize_int4: non-finite weight");
+  std::fesetround(FE_TONEAREST);
+  const int64_t G = K / groupsize;
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t j = 0; j < G; ++j) {
+      const float* w = W + n * K + j * groupsize;
+      double mn = w[0], mx = w[0];
+      for (int i = 1; i < groupsize; ++i) {
+        mn = std::fmin(mn, double(w[i]));
+        mx = std::fmax(mx, double(w[i]));
+      }
+      double z = bf16_floor(mn);
+      double s = bf16_ceil((mx - z) / 15.0);
+      if (std::fabs(z) > kBf16Max || s > kBf16Max)
+        return set_error(WQ_ERR_RANGE, "wq_quantize_int4: bf16 scale/zero overflow");
+      s_bf16[n * G + j] = bf16_bits_of(s);
+      z_bf16[n * G + j] = bf16_bits_of(z);
+      for (int i = 0; i < groupsize; ++i) {
+        double v = s == 0.0 ? 0.0 : std::nearbyint((double(w[i]) - z) / s);
+        v = v > 15.0 ? 15.0 : (v < 0.0 ? 0.0 : v);
+        q[n * K + j * groupsize + i] = uint8_t(v);
+      }
+    }
+  }
+  return ok();
+}
+
+// Nearest e3m2 code for r >= 0 (ties to even code), saturating at 28 (code 31).
+// Binade by binade: below 1/4 the spacing is 1/16 and the code is round(16 r);
+// in binade e (1..7) the spacing is 2^(e-3)/4 and the code is 4e + round(r/spacing) - 4,
+// which carries into the next binade when the rounding reaches the binade's top.
+static uint8_t e3m2_code_of(double r) {
+  if (r >= 28.0) return 31;
+  if (r < 0.25) return uint8_t(std::nearbyint(r * 16.0));  // 0..4, 4 is the first normal
+  int e = std::ilogb(r) + 3;                                 // r in [2^(e-3), 2^(e-2))
+  double n = std::nearbyint(std::ldexp(r, 5 - e));           // r / (2^(e-3)/4), in [4, 8]
+  return uint8_t(4 * e + int(n) - 4);
+}
+
+wq_status wq_quantize_fp6(const float* W, int64_t N, int64_t K, uint8_t* code, uint16_t* s_fp16) {
+  if (!W || !code || !s_fp16) return set_error(WQ_ERR_NULL, "wq_quantize_fp6: null pointer");
+  if (N < 0 || K < 0) return set_error(WQ_ERR_SHAPE, "wq_quantize_fp6: negative shape");
+  if (!all_finite(W, N * K)) return set_error(WQ_ERR_RANGE, "wq_quantize_fp6: non-finite weight");
+  std::fesetround(FE_TONEAREST);
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    double amax = 0.0;
+    for (int64_t k = 0; k < K; ++k) amax = std::fmax(amax, std::fabs(double(w[k])));
+    double s = fp16_rne_pos(amax / 28.0);
+    if (std::isinf(s)) return set_error(WQ_ERR_RANGE, "wq_quantize_fp6: fp16 scale overflow in row %lld", (long long)n);
+    s_fp16[n] = fp16_bits_of(s);
+    for (int64_t k = 0; k < K; ++k) {
+      if (s == 0.0) {
+        code[n * K + k] = 0;
+        continue;
+      }
+      double r = double(w[k]) / s;
+      uint8_t c = e3m2_code_of(std::fabs(r));
+      if (c != 0 && r < 0) c |= 0x20;
+      code[n * K + k] = c;
+    }
+  }
+  return ok();
+}
+
+wq_status wq_pack_int8(const int8_t* q, int64_t N, int64_t K, void* packed) {
+  if (!q || !packed) return set_error(WQ_ERR_NULL, "wq_pack_int8: null pointer");
+  if (N < 0 || K < 0 || K % 64) return set_error(WQ_ERR_SHAPE, "wq_pack_int8: need N, K >= 0 and K %% 64 == 0");
+  uint8_t* out = static_cast<uint8_t*>(packed);
+  for (int64_t i = 0; i < N * K; ++i) out[i] = uint8_t(int(q[i]) + 128);
+  return ok();
+}
+
+wq_status wq_pack_int4(const uint8_t* q, int64_t N, int64_t K, void* packed) {
+  if (!q || !packed) return set_error(WQ_ERR_NULL, "wq_pack_int4: null pointer");
+  if (N < 0 || K < 0 || K % 64) return set_error(WQ_ERR_SHAPE, "wq_pack_int4: need N, K >= 0 and K %% 64 == 0");
+  for (int64_t i = 0; i < N * K; ++i)
+    if (q[i] > 15) return set_error(WQ_ERR_RANGE, "wq_pack_int4: code %d > 15 at %lld", int(q[i]), (long long)i);
+  uint8_t* out = static_cast<uint8_t*>(packed);
+  for (int64_t i = 0; i < N * K; i += 2) out[i / 2] = uint8_t(q[i] | (q[i + 1] << 4));
+  return ok();
+}
+
+// Bit placement of the FP6 planes (see wq_prepack_fp6 in include/wq.h).
+static const int kRot2[8] = {0, 1, 4, 5, 8, 9, 12, 13};
+
+wq_status wq_prepack_fp6(const uint8_t* code, int64_t N, int64_t K, void* packed) {
+  if (!code || !packed) return set_error(WQ_ERR_NULL, "wq_prepack_fp6: null pointer");
+  if (N < 0 || K < 0 || K % 64) return set_error(WQ_ERR_SHAPE, "wq_prepack_fp6: need N, K >= 0 and K %% 64 == 0");
+  for (int64_t i = 0; i < N * K; ++i)
+    if (code[i] > 63) return set_error(WQ_ERR_RANGE, "wq_prepack_fp6: code %d > 63 at %lld", int(code[i]), (long long)i);
+  uint8_t* p2 = static_cast<uint8_t*>(packed);
+  uint8_t* p4 = p2 + size_t(N) * size_t(K) / 4;
+  for (int64_t n = 0; n < N; ++n) {
+    const uint8_t* c = code + n * K;
+    // 4-bit plane: one 32-bit word per 8 weights.
+    for (int64_t t = 0; t < K / 8; ++t) {
+      uint32_t w = 0;
+      for (int i = 0; i < 8; ++i) {
+        const int j = i & 3, h = i >> 2;
+        const uint32_t four = c[8 * t + i] & 0xF;
+        const int pos = (5 + 16 * h - 4 * j) & 31;
+        w |= (four << pos) | (pos > 28 ? four >> (32 - pos) : 0u);  // 4-bit field, wraps past bit 31
+      }
+      std::memcpy(p4 + n * K / 2 + 4 * t, &w, 4);
+    }
+    // 2-bit plane: one 32-bit word per 16 weights.
+    for (int64_t u = 0; u < K / 16; ++u) {
+      uint32_t w = 0;
+      for (int i = 0; i < 16; ++i) {
+        const int cc = i >> 3, j = i & 3, h = (i >> 2) & 1;
+        const int T = kRot2[4 * cc + j];
+        const uint32_t v = c[16 * u + i];
+        const uint32_t sign = (v >> 5) & 1, e2 = (v >> 4) & 1;
+        w |= sign << ((15 + 16 * h - T) & 31);
+        w |= e2 << ((9 + 16 * h - T) & 31);
+      }
+      std::memcpy(p2 + n * K / 4 + 4 * u, &w, 4);
+    }
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -22,7 +22,8 @@
  *     memory of the current device, 16-byte aligned (checked: WQ_ERR_ALIGN).
  *   - Matrices are row-major.  Scales and zeros are passed as raw 16-bit patterns
  *     (uint16_t): fp16 for int8 and FP6, bf16 for int4.
- *   - Shapes: N >= 0, M in [0, 32], K >= 0 with K % 64 == 0; int4 also needs a
+ *   - Shapes: N >= 0, M in [0, 32], 0 <= K <= 262144 with K % 64 == 0, N * K < 2^31;
+ *     int4 also needs a
  *     group size g in {32, 64, 128} with K % g == 0.  M == 0 or N == 0 is a no-op.
  *     K == 0 writes y = 0 (empty sum).
  */

@@ -1,0 +1,127 @@
+"""GPU parity: wq_linear against the fp64 oracle on seeded inputs.
+
+Sizes span several row blocks and a ragged tail in both N and K (N = 700,
+K = 2176 = 2 chunks of 1024 + 128, or 8.5 chunks of 256), every M the ABI
+accepts in groups, every format and int4 group size.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import gemm_wq_linear_b200 as wq
+import workloads
+from oracle import linear, rounding
+from wq_cases import compare, gpu_linear, oracle_weights, product_weight, x_bits
+
+pytestmark = pytest.mark.gpu
+
+N_SMALL, K_SMALL = 700, 2176
+VARIANTS = [("int8", 0), ("int4", 32), ("int4", 64), ("int4", 128), ("fp6", 0), ("bf16", 0)]
+MS = [1, 2, 3, 4, 5, 8, 16, 32]
+
+_cache = {}
+
+
+def _case(fmt, g):
+    key = (fmt, g)
+    if key not in _cache:
+        W = workloads.weights(N_SMALL, K_SMALL, seed=100 + 7 * VARIANTS.index(key))
+        _cache[key] = (oracle_weights(fmt, W.numpy(), g), product_weight(fmt, W, g))
+    return _cache[key]
+
+
+@pytest.mark.parametrize("fmt,g", VARIANTS)
+@pytest.mark.parametrize("M", MS)
+def test_linear_matches_oracle(fmt, g, M):
+    Wd, pw = _case(fmt, g)
+    x = workloads.activations(M, K_SMALL, seed=1000 + M)
+    y = gpu_linear(x, pw)
+    y_ref = linear.linear_ref(x_bits(x), Wd)
+    compare(y, y_ref)
+
+
+@pytest.mark.parametrize("fmt,g", VARIANTS)
+def test_linear_pdl_flag_same_result(fmt, g):
+    Wd, pw = _case(fmt, g)
+    x = workloads.activations(2, K_SMALL, seed=77).cuda()
+    y0 = wq.linear(x, pw)
+    y1 = wq.linear(x, pw, flags=wq.WQ_LAUNCH_PDL)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+
+
+def _exact_case(fmt, g, M, N, K, seed):
+    """Integer activations, power-of-two scales: every partial sum is exact in fp32,
+    so the kernel's bf16 output must equal RNE_bf16 of the exact result bit for bit."""
+    gen = workloads.generator(seed)
+    x = workloads.integer_activations(M, K, seed)
+    if fmt == "int8":
+        q = torch.randint(-127, 128, (N, K), generator=gen, dtype=torch.int8)
+        s = torch.full((N,), 0x2C00, dtype=torch.int16)  # fp16 2^-4
+        pw = wq.PackedWeight.from_codes("int8", q, s)
+        Wd = linear.deq_weights("int8", q.numpy(), s.numpy().view(np.uint16))
+    elif fmt == "int4":
+        q = torch.randint(0, 16, (N, K), generator=gen, dtype=torch.uint8)
+        s = torch.full((N, K // g), 0x3D80, dtype=torch.int16)  # bf16 2^-4
+        z = torch.full((N, K // g), int(np.int16(np.uint16(0xBF00))), dtype=torch.int16)  # bf16 -0.5
+        pw = wq.PackedWeight.from_codes("int4", q, s, z, g)
+        Wd = linear.deq_weights("int4", q.numpy(), s.numpy().view(np.uint16), z.numpy().view(np.uint16), g)
+    elif fmt == "fp6":
+        c = torch.randint(0, 64, (N, K), generator=gen, dtype=torch.uint8)
+        s = torch.full((N,), 0x3800, dtype=torch.int16)  # fp16 0.5
+        pw = wq.PackedWeight.from_codes("fp6", c, s)
+        Wd = linear.deq_weights("fp6", c.numpy(), s.numpy().view(np.uint16))
+    else:
+        w = torch.randint(-16, 17, (N, K), generator=gen).to(torch.bfloat16)
+        pw = wq.PackedWeight.from_codes("bf16", w.view(torch.int16))
+        Wd = linear.deq_weights("bf16", w.view(torch.int16).numpy().view(np.uint16))
+    return x, pw, Wd
+
+
+@pytest.mark.parametrize("fmt,g", VARIANTS)
+@pytest.mark.parametrize("M", [1, 3, 4, 8, 32])
+def test_linear_exact_integer_inputs_bit_identical(fmt, g, M):
+    N, K = 300, 1152
+    x, pw, Wd = _exact_case(fmt, g, M, N, K, seed=5 + M)
+    y = gpu_linear(x, pw)
+    ref_bits = rounding.bf16_bits(rounding.bf16_rne(linear.linear_ref(x_bits(x), Wd)))
+    got = y.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref_bits)
+
+
+@pytest.mark.parametrize("fmt,g", [("int8", 0), ("int4", 32), ("fp6", 0), ("bf16", 0)])
+def test_linear_degenerate_shapes(fmt, g):
+    # N = 1 (one output row), K = 64 (one partial chunk), M = 1
+    for (M, N, K) in [(1, 1, 64), (2, 5, 128), (4, 129, 64)]:
+        W = workloads.weights(N, K, seed=3)
+        pw = product_weight(fmt, W, g if K % max(g, 1) == 0 else 32)
+        x = workloads.activations(M, K, seed=4)
+        Wd = oracle_weights(fmt, W.numpy(), g if K % max(g, 1) == 0 else 32)
+        compare(gpu_linear(x, pw), linear.linear_ref(x_bits(x), Wd))
+
+
+def test_linear_k_zero_writes_zeros():
+    y = torch.full((2, 16), 7.0, dtype=torch.bfloat16, device="cuda")
+    x = torch.empty(2, 0, dtype=torch.bfloat16, device="cuda")
+    p = torch.empty(16, dtype=torch.uint8, device="cuda")
+    s = torch.empty(16, dtype=torch.int16, device="cuda")
+    wq.wq_linear(x, p, s, None, y, 2, 16, 0, "int8")
+    torch.cuda.synchronize()
+    assert torch.all(y == 0)
+
+
+def test_linear_zero_weight_rows():
+    W = workloads.weights(256, 512, seed=9)
+    W[17] = 0.0
+    W[200] = 0.0
+    for fmt, g in [("int8", 0), ("int4", 64), ("fp6", 0)]:
+        pw = product_weight(fmt, W, g)
+        x = workloads.activations(2, 512, seed=10)
+        y = gpu_linear(x, pw)
+        assert torch.all(y[:, 17] == 0) and torch.all(y[:, 200] == 0)
+        compare(y, linear.linear_ref(x_bits(x), oracle_weights(fmt, W.numpy(), g)))
+
+
+def test_sync_status_ok():
+    wq.wq_sync_status()

@@ -1,0 +1,231 @@
+"""Host-side checks of libwq (no GPU needed): exports, sizes, quantizers and
+packers against the oracle, and argument validation of the compute entry points.
+"""
+
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import gemm_wq_linear_b200 as wq
+import workloads
+from oracle import formats, layout
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _np(t):
+    return t.numpy()
+
+
+def _u16(t):
+    return t.numpy().view(np.uint16)
+
+
+# ------------------------------------------------------------------ ABI surface
+def test_library_exports_every_declared_function():
+    with open(os.path.join(ROOT, "include", "wq.h")) as f:
+        src = f.read()
+    declared = set(re.findall(r"^\s*(?:const\s+)?[\w\*\s]+?\b(wq_\w+)\s*\(", src, flags=re.M))
+    assert declared, "no declarations parsed"
+    for name in sorted(declared):
+        assert hasattr(wq.lib, name), name
+    assert set(wq.EXPORTS) == declared
+
+
+def test_sizes():
+    assert wq.wq_packed_size("int8", 10, 64) == 640
+    assert wq.wq_packed_size("int4", 10, 64) == 320
+    assert wq.wq_packed_size("fp6", 10, 64) == 480
+    assert wq.wq_packed_size("bf16", 10, 64) == 1280
+    assert wq.wq_packed_size(9, 10, 64) == 0
+    assert wq.wq_scales_size("int8", 10, 64) == 20
+    assert wq.wq_scales_size("fp6", 10, 64) == 20
+    assert wq.wq_scales_size("int4", 10, 256, 64) == 10 * 4 * 2
+    assert wq.wq_scales_size("int4", 10, 256, 48) == 0
+    assert wq.wq_scales_size("bf16", 10, 64) == 0
+    assert wq.wq_version().startswith("wq ")
+
+
+# ------------------------------------------------------------------ quantizers
+@pytest.mark.parametrize("seed", [0, 1])
+def test_quantize_int8_matches_oracle(seed):
+    W = workloads.weights(48, 1024, seed)
+    q, s = wq.wq_quantize_int8(W)
+    qo, so = formats.quantize_int8(W.numpy())
+    assert np.array_equal(_np(q), qo)
+    assert np.array_equal(_u16(s), so)
+
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_quantize_int4_matches_oracle(g):
+    W = workloads.weights(40, 1024, 3)
+    q, s, z = wq.wq_quantize_int4(W, g)
+    qo, so, zo = formats.quantize_int4(W.numpy(), g)
+    assert np.array_equal(_np(q), qo)
+    assert np.array_equal(_u16(s), so)
+    assert np.array_equal(_u16(z), zo)
+
+
+def test_quantize_fp6_matches_oracle():
+    W = workloads.weights(64, 1024, 4)
+    c, s = wq.wq_quantize_fp6(W)
+    co, so = formats.quantize_fp6(W.numpy())
+    assert np.array_equal(_np(c), co)
+    assert np.array_equal(_u16(s), so)
+
+
+def test_quantizers_on_ties_and_edges():
+    # rows built so that W / s lands exactly on e3m2 / integer midpoints
+    s = 1311 * 2.0 ** -17  # fp16 scale of a row whose max is 28 * s (FP6) / 127 * s (int8)
+    mids = [0.03125, 0.09375, 0.21875, 0.40625, 2.25, 5.5, 13.0, 26.0, 27.9, 0.5, 1.125]
+    row = np.array([28.0] + mids + [-m for m in mids] + [0.0] * 41, dtype=np.float64) * s
+    W = torch.from_numpy(row.astype(np.float32)[None, :].repeat(3, axis=0).copy())
+    c, sb = wq.wq_quantize_fp6(W)
+    co, sbo = formats.quantize_fp6(W.numpy())
+    assert np.array_equal(_np(c), co) and np.array_equal(_u16(sb), sbo)
+    row8 = np.array([127.0, 0.5, 1.5, 2.5, -0.5, -1.5, 126.5] + [0.0] * 57) * s
+    W8 = torch.from_numpy(row8.astype(np.float32)[None, :].copy())
+    q, sb = wq.wq_quantize_int8(W8)
+    qo, sbo = formats.quantize_int8(W8.numpy())
+    assert np.array_equal(_np(q), qo) and np.array_equal(_u16(sb), sbo)
+    # zero rows, constant groups, tiny values (fp16 subnormal scales)
+    Wz = torch.zeros(2, 128)
+    Wz[1] = 3e-6
+    for g in (32, 64):
+        a = wq.wq_quantize_int4(Wz, g)
+        b = formats.quantize_int4(Wz.numpy(), g)
+        assert all(np.array_equal(_np(x) if x.dtype != torch.int16 else _u16(x), y) for x, y in zip(a, b))
+    a = wq.wq_quantize_int8(Wz)
+    b = formats.quantize_int8(Wz.numpy())
+    assert np.array_equal(_np(a[0]), b[0]) and np.array_equal(_u16(a[1]), b[1])
+    a = wq.wq_quantize_fp6(Wz)
+    b = formats.quantize_fp6(Wz.numpy())
+    assert np.array_equal(_np(a[0]), b[0]) and np.array_equal(_u16(a[1]), b[1])
+
+
+def test_quantizer_errors():
+    W = torch.zeros(2, 64)
+    W[0, 0] = float("nan")
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_quantize_int8(W)
+    assert e.value.status == 7
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_quantize_int4(torch.zeros(2, 64), 48)
+    assert e.value.status == 4
+    big = torch.full((1, 64), 3e38)
+    with pytest.raises(wq.WQError):
+        wq.wq_quantize_int8(big)  # fp16 scale overflow
+
+
+# ------------------------------------------------------------------ packers
+def _codes(kind, N, K, seed):
+    lo, hi = {"int8": (-127, 127), "int4": (0, 15), "fp6": (0, 63)}[kind]
+    dt = {"int8": torch.int8, "int4": torch.uint8, "fp6": torch.uint8}[kind]
+    return workloads.random_codes((N, K), lo, hi, seed).to(dt)
+
+
+def _pack(kind, c):
+    return {"int8": wq.wq_pack_int8, "int4": wq.wq_pack_int4, "fp6": wq.wq_prepack_fp6}[kind](c)
+
+
+def _unpack(kind, p, N, K):
+    return {"int8": layout.unpack_int8, "int4": layout.unpack_int4, "fp6": layout.unpack_fp6}[kind](p.numpy(), N, K)
+
+
+@pytest.mark.parametrize("kind", ["int8", "int4", "fp6"])
+def test_pack_unpack_identity_random(kind):
+    N, K = 3, 128
+    c = _codes(kind, N, K, 21)
+    p = _pack(kind, c)
+    assert p.numel() == wq.wq_packed_size(kind, N, K)
+    assert np.array_equal(_unpack(kind, p, N, K), c.numpy())
+
+
+@pytest.mark.parametrize("kind", ["int8", "int4", "fp6"])
+def test_pack_one_hot_every_position(kind):
+    """A single nonzero code at each position must come back at that position only."""
+    N, K = 2, 64
+    val = {"int8": 127, "int4": 15, "fp6": 63}[kind]
+    dt = torch.int8 if kind == "int8" else torch.uint8
+    for pos in range(N * K):
+        c = torch.zeros(N, K, dtype=dt)
+        c.view(-1)[pos] = val
+        got = _unpack(kind, _pack(kind, c), N, K)
+        assert np.array_equal(got, c.numpy()), (kind, pos)
+
+
+@pytest.mark.parametrize("kind", ["int8", "int4", "fp6"])
+def test_pack_constant_codes(kind):
+    N, K = 2, 64
+    dt = torch.int8 if kind == "int8" else torch.uint8
+    for v in {"int8": (0, -127, 127), "int4": (0, 15), "fp6": (0, 32, 31, 63)}[kind]:
+        c = torch.full((N, K), v, dtype=dt)
+        assert np.array_equal(_unpack(kind, _pack(kind, c), N, K), c.numpy())
+
+
+def test_pack_errors():
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_pack_int4(torch.full((1, 64), 16, dtype=torch.uint8))
+    assert e.value.status == 7
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_prepack_fp6(torch.full((1, 64), 64, dtype=torch.uint8))
+    assert e.value.status == 7
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_pack_int8(torch.zeros(1, 96, dtype=torch.int8))
+    assert e.value.status == 2
+
+
+# ------------------------------------------------------------------ argument validation (no launch)
+class _FakePtr:
+    """Stands in for a tensor: only data_ptr() is read by the binding."""
+
+    def __init__(self, addr):
+        self.addr = addr
+
+    def data_ptr(self):
+        return self.addr
+
+
+A = _FakePtr(0x10000)  # aligned, never dereferenced: validation fails first
+
+
+def _lin(**kw):
+    args = dict(x=A, packed=A, scales=A, zeros=None, y=A, M=1, N=128, K=128, fmt="int8", groupsize=0)
+    args.update(kw)
+    wq.wq_linear(**args, stream=0)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(fmt=7), 3),
+    (dict(M=33), 2),
+    (dict(M=-1), 2),
+    (dict(K=96), 2),
+    (dict(N=-5), 2),
+    (dict(fmt="int4", zeros=A, groupsize=48), 4),
+    (dict(fmt="int4", zeros=A, groupsize=256), 4),
+    (dict(fmt="int4", zeros=A, groupsize=128, K=192), 4),
+    (dict(x=None), 1),
+    (dict(scales=None), 1),
+    (dict(fmt="int4", groupsize=32), 1),          # zeros missing
+    (dict(zeros=A), 1),                           # zeros given for int8
+    (dict(fmt="bf16"), 1),                        # scales given for bf16
+    (dict(x=_FakePtr(0x10008)), 5),
+    (dict(y=_FakePtr(0x10002)), 5),
+    (dict(scales=_FakePtr(0x10004)), 5),
+])
+def test_linear_rejects_bad_arguments(kw, status):
+    with pytest.raises(wq.WQError) as e:
+        _lin(**kw)
+    assert e.value.status == status
+    assert wq.lib.wq_last_error().decode() != ""
+
+
+def test_linear_empty_is_noop():
+    _lin(M=0)  # no launch, no pointer use
+    _lin(N=0, x=None, packed=None, y=None, scales=None)
+    wq.wq_linear_ex(A, A, A, None, A, 0, 128, 128, "int8", 0, 0, flags=wq.WQ_LAUNCH_PDL)
+    with pytest.raises(wq.WQError):
+        wq.wq_linear_ex(A, A, A, None, A, 1, 128, 128, "int8", 0, 0, flags=0x8)

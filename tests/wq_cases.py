@@ -1,0 +1,70 @@
+"""Shared helpers of the GPU parity tests: build one seeded case on both sides.
+
+The product side quantizes and packs with libwq and runs the CUDA kernels; the
+oracle side quantizes the same seeded float32 weights with ``oracle.formats``
+and computes ``oracle.linear``.  The two never exchange codes or results.
+"""
+
+import numpy as np
+import torch
+
+import gemm_wq_linear_b200 as wq
+import workloads
+from oracle import formats, linear, rounding
+
+FMTS = ("int8", "int4", "fp6", "bf16")
+
+# Output tolerance (fp32 accumulation, one bf16 rounding of the result):
+# rel-L2 against the bf16-rounded fp64 result, and per element against the
+# unrounded fp64 result.
+REL_L2 = 1e-3
+ELEM_ABS = 1e-2
+
+
+def oracle_weights(fmt, Wnp, g=0):
+    """Oracle quantization + dequantization of float32 W (numpy) -> float64 deq W."""
+    if fmt == "int8":
+        q, s = formats.quantize_int8(Wnp)
+        return linear.deq_weights("int8", q, s)
+    if fmt == "int4":
+        q, s, z = formats.quantize_int4(Wnp, g)
+        return linear.deq_weights("int4", q, s, z, g)
+    if fmt == "fp6":
+        c, s = formats.quantize_fp6(Wnp)
+        return linear.deq_weights("fp6", c, s)
+    bits = rounding.bf16_bits(rounding.bf16_rne(Wnp.astype(np.float64)))
+    return linear.deq_weights("bf16", bits)
+
+
+def product_weight(fmt, W, g=0):
+    """libwq quantization + packing of float32 W (CPU torch) -> device PackedWeight."""
+    return wq.PackedWeight.quantize(W, fmt, g)
+
+
+def x_bits(x):
+    return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def gpu_linear(x, pw, flags=0):
+    y = wq.linear(x.cuda(), pw, flags=flags)
+    torch.cuda.synchronize()
+    return y.cpu()
+
+
+def compare(y_gpu, y_ref):
+    """Assert the tolerance; return (rel_l2_vs_rounded, rel_l2_vs_fp64, max_elem_ratio)."""
+    yg = y_gpu.to(torch.float64).numpy()
+    rb = rounding.bf16_rne(y_ref)
+    den = np.linalg.norm(rb)
+    rel = np.linalg.norm(yg - rb) / den if den > 0 else np.linalg.norm(yg - rb)
+    rel64 = np.linalg.norm(yg - y_ref) / max(np.linalg.norm(y_ref), 1e-300)
+    ratio = np.max(np.abs(yg - y_ref) / (ELEM_ABS * (np.abs(y_ref) + 1.0))) if yg.size else 0.0
+    assert rel <= REL_L2, f"rel-L2 {rel:.3e} > {REL_L2}"
+    assert ratio <= 1.0, f"per-element error ratio {ratio:.3f} > 1"
+    return rel, rel64, ratio
+
+
+def make_case(fmt, M, N, K, g=0, seed=0, xseed=None):
+    W = workloads.weights(N, K, seed)
+    x = workloads.activations(M, K, seed + 7 if xseed is None else xseed)
+    return W, x
