@@ -11,8 +11,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libwq.so")
-SOURCES = ["wq_host.cpp", "wq_device.cu", "wq_gemv.cu"]
-HEADERS = ["wq_internal.h", "wq_kernels.cuh", "decode.cuh"]
+SOURCES = ["wq_host.cpp", "wq_device.cu", "wq_gemv.cu", "wq_gemm_sm100.cu"]
+HEADERS = ["wq_internal.h", "wq_kernels.cuh", "decode.cuh", "ptx.cuh", "tcgen05.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",

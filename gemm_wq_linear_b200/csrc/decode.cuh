@@ -6,9 +6,8 @@
 // "重新设计内核方案": dequantize inside registers with bit-level parallelism and
 // splice the 2-bit and 4-bit pieces of each 6-bit weight in parallel).
 //
-// Pair convention: a decoded pair register holds (lo, hi) = (k, k + 4) of an
-// 8-weight group for int4 and FP6, so the activations are permuted the same way
-// once per chunk instead of permuting every weight.
+// Pair convention: a decoded pair register holds (lo, hi) = (k, k + 1); the
+// packers place the codes inside each word so that this needs no permutation.
 #pragma once
 #include <cstdint>
 
@@ -20,8 +19,8 @@ constexpr uint32_t kBf16Magic128x2 = 0x43004300u;
 
 __device__ __forceinline__ uint32_t rotl32(uint32_t x, int s) { return __funnelshift_l(x, x, s); }
 
-// int4: word w holds q[8t + i] in bits 4i..4i+3.  Output p[r] = bf16 pair
-// (128 + q[8t + r], 128 + q[8t + r + 4]), r = 0..3.
+// int4: word w holds q[8t + 2r + h] in bits 4r + 16h .. +3.  Output p[r] = bf16
+// pair (128 + q[8t + 2r], 128 + q[8t + 2r + 1]), r = 0..3.
 __device__ __forceinline__ void decode_int4_word(uint32_t w, uint32_t p[4]) {
   p[0] = (w & 0x000F000Fu) | kBf16Magic128x2;
   p[1] = ((w >> 4) & 0x000F000Fu) | kBf16Magic128x2;
@@ -31,7 +30,7 @@ __device__ __forceinline__ void decode_int4_word(uint32_t w, uint32_t p[4]) {
 
 // FP6 (2+4 planes): p2 is the 2-bit-plane word of 16 weights, p4a / p4b the two
 // 4-bit-plane words of its first and second 8 weights.  Output p[4c + j] = bf16
-// pair (k = 8c + j, 8c + j + 4) holding code value * 2^-124 (subnormal for e = 0).
+// pair (k = 8c + 2j, 8c + 2j + 1) holding code value * 2^-124 (subnormal for e = 0).
 __device__ __forceinline__ void decode_fp6_words(uint32_t p2, uint32_t p4a, uint32_t p4b, uint32_t p[8]) {
   constexpr uint32_t kFour = 0x01E001E0u;  // bits 5..8 of each half: (e1 e0 m1 m0)
   constexpr uint32_t kTwo = 0x82008200u;   // bits 15 and 9 of each half: sign, e2
@@ -80,6 +79,19 @@ __device__ __forceinline__ void fma_bf16x2(float& acc, uint32_t a, uint32_t b) {
   fma_bf16_hi(acc, a, b);
 }
 
+// (acc0, acc1) += (w0 * x0, w1 * x1): packed fp32 FMA of sm_100 (one
+// instruction for two lanes), each product rounded once into its accumulator.
+__device__ __forceinline__ void ffma2(float& acc0, float& acc1, float w0, float w1, float x0, float x1) {
+  asm("{.reg .b64 a, w, x;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "mov.b64 w, {%2, %3};\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "fma.rn.f32x2 a, w, x, a;\n\t"
+      "mov.b64 {%0, %1}, a;}\n"
+      : "+f"(acc0), "+f"(acc1)
+      : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
+}
+
 // Exact bf16 pair -> two floats.
 __device__ __forceinline__ float bf16_lo_f(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
@@ -91,8 +103,5 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   return r;
 }
 
-// (a.lo, b.lo) and (a.hi, b.hi) recombined: used to permute activation pairs.
-__device__ __forceinline__ uint32_t pair_lo(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x5410); }
-__device__ __forceinline__ uint32_t pair_hi(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x7632); }
 
 }  // namespace wq

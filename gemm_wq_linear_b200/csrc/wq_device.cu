@@ -4,11 +4,50 @@
 #include "wq_kernels.cuh"
 #include "decode.cuh"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 namespace wq {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
+                         uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, int swizzle_bytes) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_u32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                             uint32_t box_inner, uint32_t box_rows) {
+  return make_tmap_2d(map, base, 4, inner, rows, row_bytes, box_inner, box_rows, 0);
+}
 
 // Number of SMs of each device, cached (cudaDeviceGetAttribute is cheap but
 // this keeps wq_linear free of any query on the hot path).
@@ -27,7 +66,9 @@ static int sm_count_of_current_device() {
 }
 
 // Largest K: bounds the per-CTA shared memory of the GEMV partial sums.
-static const int kMaxK = 262144;
+static const int kMaxK = 65536;
+// Largest M served by the CUDA-core GEMV; larger M runs the tcgen05 GEMM.
+static const int kGemvMaxM = 4;
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -50,8 +91,8 @@ __global__ void unpack_debug_kernel(const uint8_t* __restrict__ packed, int fmt,
       uint32_t p[4];
       decode_int4_word(words[q], p);
       for (int r = 0; r < 4; ++r) {
-        v[8 * q + r] = bf16_lo_f(p[r]) - 128.f;
-        v[8 * q + r + 4] = bf16_hi_f(p[r]) - 128.f;
+        v[8 * q + 2 * r] = bf16_lo_f(p[r]) - 128.f;
+        v[8 * q + 2 * r + 1] = bf16_hi_f(p[r]) - 128.f;
       }
     }
   } else if (fmt == WQ_FP6_E3M2) {
@@ -72,8 +113,8 @@ __global__ void unpack_debug_kernel(const uint8_t* __restrict__ packed, int fmt,
           float lo = 0.f, hi = 0.f;
           fma_bf16_lo(lo, p[4 * c + j], one);
           fma_bf16_hi(hi, p[4 * c + j], one);
-          v[16 * u + 8 * c + j] = lo * 0x1p124f;
-          v[16 * u + 8 * c + j + 4] = hi * 0x1p124f;
+          v[16 * u + 8 * c + 2 * j] = lo * 0x1p124f;
+          v[16 * u + 8 * c + 2 * j + 1] = hi * 0x1p124f;
         }
     }
   } else if (fmt == WQ_INT8) {
@@ -135,7 +176,15 @@ wq_status wq_linear_ex(const void* x, const void* packed, const void* scales, co
   if (st != WQ_OK) return st;
   if (flags & ~WQ_LAUNCH_PDL) return set_error(WQ_ERR_SHAPE, "%s: unknown flags 0x%x", fn, flags);
   if (M == 0 || N == 0) return ok();
-  if (!x || !packed || !y) return set_error(WQ_ERR_NULL, "%s: x, packed and y must be non-null", fn);
+  if (!y) return set_error(WQ_ERR_NULL, "%s: y must be non-null", fn);
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (K == 0) {  // empty sum: x, packed, scales are not read
+    if (!aligned16(y)) return set_error(WQ_ERR_ALIGN, "%s: device pointers must be 16-byte aligned", fn);
+    cudaError_t e = cudaMemsetAsync(y, 0, size_t(M) * size_t(N) * 2, stream);
+    if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+    return ok();
+  }
+  if (!x || !packed) return set_error(WQ_ERR_NULL, "%s: x, packed and y must be non-null", fn);
   if (fmt != WQ_BF16 && !scales) return set_error(WQ_ERR_NULL, "%s: scales must be non-null", fn);
   if (fmt == WQ_BF16 && scales) return set_error(WQ_ERR_NULL, "%s: scales must be NULL for bf16 weights", fn);
   if ((fmt == WQ_INT4) != (zeros != nullptr))
@@ -143,29 +192,39 @@ wq_status wq_linear_ex(const void* x, const void* packed, const void* scales, co
   if (!aligned16(x) || !aligned16(packed) || !aligned16(y) || (scales && !aligned16(scales)) ||
       (zeros && !aligned16(zeros)))
     return set_error(WQ_ERR_ALIGN, "%s: device pointers must be 16-byte aligned", fn);
-  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-  if (K == 0) {
-    cudaError_t e = cudaMemsetAsync(y, 0, size_t(M) * size_t(N) * 2, stream);
-    if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  const int sms = sm_count_of_current_device();
+  const int pdl = (flags & WQ_LAUNCH_PDL) ? 1 : 0;
+  if (M <= kGemvMaxM) {
+    GemvParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.packed = packed;
+    p.scales = static_cast<const uint16_t*>(scales);
+    p.zeros = static_cast<const uint16_t*>(zeros);
+    p.y = static_cast<uint16_t*>(y);
+    p.M = int(M);
+    p.N = int(N);
+    p.K = int(K);
+    p.groupsize = groupsize;
+    p.fmt = fmt;
+    p.pdl = pdl;
+    cudaError_t e = launch_gemv(p, stream, sms);
+    if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "%s: GEMV launch failed: %s", fn, cudaGetErrorString(e));
     return ok();
   }
-  const int sms = sm_count_of_current_device();
-  GemvParams p{};
+  GemmParams p{};
+  p.x = static_cast<const uint16_t*>(x);
   p.packed = packed;
   p.scales = static_cast<const uint16_t*>(scales);
   p.zeros = static_cast<const uint16_t*>(zeros);
+  p.y = static_cast<uint16_t*>(y);
+  p.M = int(M);
   p.N = int(N);
   p.K = int(K);
   p.groupsize = groupsize;
   p.fmt = fmt;
-  p.pdl = (flags & WQ_LAUNCH_PDL) ? 1 : 0;
-  for (int64_t m0 = 0; m0 < M; m0 += 4) {
-    p.M = int(M - m0 < 4 ? M - m0 : 4);
-    p.x = static_cast<const uint16_t*>(x) + m0 * K;
-    p.y = static_cast<uint16_t*>(y) + m0 * N;
-    cudaError_t e = launch_gemv(p, stream, sms);
-    if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
-  }
+  p.pdl = pdl;
+  cudaError_t e = launch_gemm(p, stream, sms);
+  if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "%s: tensor-core GEMM launch failed: %s", fn, cudaGetErrorString(e));
   return ok();
 }
 
@@ -190,6 +249,12 @@ wq_status wq_unpack_debug(const void* packed, int fmt, int64_t N, int64_t K, voi
 wq_status wq_sync_status(void* cuda_stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "wq_sync_status: %s", cudaGetErrorString(e));
+  uint32_t st = 0, st2 = 0;
+  e = gemv_take_status(&st);
+  if (e == cudaSuccess) e = gemm_take_status(&st2);
+  if (e != cudaSuccess) return set_error(WQ_ERR_CUDA, "wq_sync_status: %s", cudaGetErrorString(e));
+  st |= st2;
+  if (st) return set_error(WQ_ERR_TIMEOUT, "wq_sync_status: a device-side wait timed out (status 0x%x)", st);
   return ok();
 }
 

@@ -262,7 +262,12 @@ wq_status wq_pack_int4(const uint8_t* q, int64_t N, int64_t K, void* packed) {
   for (int64_t i = 0; i < N * K; ++i)
     if (q[i] > 15) return set_error(WQ_ERR_RANGE, "wq_pack_int4: code %d > 15 at %lld", int(q[i]), (long long)i);
   uint8_t* out = static_cast<uint8_t*>(packed);
-  for (int64_t i = 0; i < N * K; i += 2) out[i / 2] = uint8_t(q[i] | (q[i + 1] << 4));
+  // word t of a row: k = 8t + 2r + h at bits 4r + 16h (see include/wq.h)
+  for (int64_t i = 0; i < N * K; i += 8) {
+    uint32_t w = 0;
+    for (int e = 0; e < 8; ++e) w |= uint32_t(q[i + e]) << (4 * (e >> 1) + 16 * (e & 1));
+    std::memcpy(out + i / 2, &w, 4);
+  }
   return ok();
 }
 
@@ -282,7 +287,7 @@ wq_status wq_prepack_fp6(const uint8_t* code, int64_t N, int64_t K, void* packed
     for (int64_t t = 0; t < K / 8; ++t) {
       uint32_t w = 0;
       for (int i = 0; i < 8; ++i) {
-        const int j = i & 3, h = i >> 2;
+        const int j = i >> 1, h = i & 1;
         const uint32_t four = c[8 * t + i] & 0xF;
         const int pos = (5 + 16 * h - 4 * j) & 31;
         w |= (four << pos) | (pos > 28 ? four >> (32 - pos) : 0u);  // 4-bit field, wraps past bit 31
@@ -293,7 +298,7 @@ wq_status wq_prepack_fp6(const uint8_t* code, int64_t N, int64_t K, void* packed
     for (int64_t u = 0; u < K / 16; ++u) {
       uint32_t w = 0;
       for (int i = 0; i < 16; ++i) {
-        const int cc = i >> 3, j = i & 3, h = (i >> 2) & 1;
+        const int cc = i >> 3, j = (i >> 1) & 3, h = i & 1;
         const int T = kRot2[4 * cc + j];
         const uint32_t v = c[16 * u + i];
         const uint32_t sign = (v >> 5) & 1, e2 = (v >> 4) & 1;

@@ -1,11 +1,45 @@
 // Launch parameters and launchers of the wq device kernels.
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace wq {
 
+// Encodes a 2-D tensor map over a row-major matrix viewed as 32-bit elements:
+// `rows` rows of `inner` elements, rows `row_bytes` apart, copied in boxes of
+// box_inner x box_rows elements (out-of-range elements read as zero).
+cudaError_t make_tmap_u32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                             uint32_t box_inner, uint32_t box_rows);
+
+// General 2-D tensor map: elements of `elem_bytes` (4: uint32, 2: bf16), with
+// the given swizzle span in bytes (0, 32, 64 or 128).
+cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
+                         uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, int swizzle_bytes);
+
+struct GemmParams {
+  CUtensorMap tm_w;        // packed weights (FP6: the 4-bit plane; bf16: W)
+  CUtensorMap tm_w2;       // FP6: the 2-bit plane
+  CUtensorMap tm_x;        // activations, 128-byte swizzled boxes
+  const uint16_t* x;
+  const void* packed;
+  const uint16_t* scales;
+  const uint16_t* zeros;
+  uint16_t* y;
+  int M, N, K, groupsize, fmt;
+  int splits;              // CTAs of a cluster splitting K (set by the launcher)
+  int kb_per_split;        // 128-wide k-blocks per split (set by the launcher)
+  uint32_t tmem_cols;      // tensor-memory columns allocated per CTA
+  int pdl;
+};
+
+// tcgen05 swap-AB GEMM, 1 <= M <= 32 (used for M > 4).
+cudaError_t launch_gemm(const GemmParams& p, cudaStream_t s, int sm_count);
+cudaError_t gemm_take_status(uint32_t* status);
+
 struct GemvParams {
+  CUtensorMap tm_w;        // packed weights (FP6: the 4-bit plane)
+  CUtensorMap tm_w2;       // FP6: the 2-bit plane
   const uint16_t* x;       // bf16 [M, K]
   const void* packed;      // packed weights of `fmt`
   const uint16_t* scales;  // fp16 [N] (int8, FP6) or bf16 [N, K/g] (int4)
@@ -13,11 +47,16 @@ struct GemvParams {
   uint16_t* y;             // bf16 [M, N]
   int M, N, K, groupsize, fmt;
   int rows_per_cta;        // set by the launcher
+  int stages;              // shared-memory ring depth, set by the launcher
+  int box_rows;            // rows per tensor-copy box (rows_per_cta is a multiple)
   int pdl;                 // programmatic dependent launch enabled
 };
 
 // CUDA-core GEMV, 1 <= M <= 4.
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t s, int sm_count);
+
+// Reads and clears the device status word of the GEMV kernels.
+cudaError_t gemv_take_status(uint32_t* status);
 
 // Decode-only kernel: code values as bf16 [N, K].
 cudaError_t launch_unpack_debug(const void* packed, int fmt, int N, int K, uint16_t* out, cudaStream_t s);

@@ -22,7 +22,7 @@
  *     memory of the current device, 16-byte aligned (checked: WQ_ERR_ALIGN).
  *   - Matrices are row-major.  Scales and zeros are passed as raw 16-bit patterns
  *     (uint16_t): fp16 for int8 and FP6, bf16 for int4.
- *   - Shapes: N >= 0, M in [0, 32], 0 <= K <= 262144 with K % 64 == 0, N * K < 2^31;
+ *   - Shapes: N >= 0, M in [0, 32], 0 <= K <= 65536 with K % 64 == 0, N * K < 2^31;
  *     int4 also needs a
  *     group size g in {32, 64, 128} with K % g == 0.  M == 0 or N == 0 is a no-op.
  *     K == 0 writes y = 0 (empty sum).
@@ -109,8 +109,10 @@ wq_status wq_quantize_fp6(const float* W, int64_t N, int64_t K, uint8_t* code, u
  * q: int8 [N, K] in [-127, 127] (host); packed: wq_packed_size(WQ_INT8) bytes (host). */
 wq_status wq_pack_int8(const int8_t* q, int64_t N, int64_t K, void* packed);
 
-/* int4: byte n*K/2 + k/2 holds q[n,k] in its low nibble for even k, high nibble
- * for odd k.  q: uint8 [N, K] codes 0..15 (host); packed: N*K/2 bytes (host). */
+/* int4: little-endian 32-bit word t of row n (bytes n*K/2 + 4t .. +3) holds the
+ * codes of k = 8t + 2r + h (r in 0..3, h in 0..1) in bits 4r + 16h .. 4r + 16h + 3,
+ * so one mask-and-or turns (w >> 4r) into the bf16 pair (k = 8t+2r, 8t+2r+1).
+ * q: uint8 [N, K] codes 0..15 (host); packed: N*K/2 bytes (host). */
 wq_status wq_pack_int4(const uint8_t* q, int64_t N, int64_t K, void* packed);
 
 /* FP6: each code c (bit 5 sign, bits 4..2 exponent e2 e1 e0, bits 1..0 mantissa)
@@ -119,13 +121,13 @@ wq_status wq_pack_int4(const uint8_t* q, int64_t N, int64_t K, void* packed);
  * the 2-bit plane first (N*K/4 bytes, row n at byte n*K/4), then the 4-bit plane
  * (N*K/2 bytes).  Bit positions are taken
  * modulo 32 inside little-endian 32-bit words.
- *   4-bit plane: word t of row n (bytes n*K/2 + 4t .. +3) holds k = 8t + i,
- *     i = j + 4h (j in 0..3, h in 0..1); bit b (0..3) of the piece of k sits at
+ *   4-bit plane: word t of row n (bytes n*K/2 + 4t .. +3) holds k = 8t + 2j + h
+ *     (j in 0..3, h in 0..1); bit b (0..3) of the piece of k sits at
  *     bit (5 + 16h - 4j + b) mod 32.
- *   2-bit plane: word u of row n (bytes n*K/4 + 4u .. +3) holds k = 16u + i,
- *     i = 8c + j + 4h (c, h in 0..1, j in 0..3); with T = {0,1,4,5,8,9,12,13}[4c + j]
- *     the sign bit sits at (15 + 16h - T) mod 32 and e2 at (9 + 16h - T) mod 32.
- * With this permutation the kernel forms the bf16 pair (k = 8t+j, 8t+j+4) as
+ *   2-bit plane: word u of row n (bytes n*K/4 + 4u .. +3) holds k = 16u + 8c + 2j + h
+ *     (c, h in 0..1, j in 0..3); with T = {0,1,4,5,8,9,12,13}[4c + j] the sign bit
+ *     sits at (15 + 16h - T) mod 32 and e2 at (9 + 16h - T) mod 32.
+ * With this permutation the kernel forms the bf16 pair (k = 8t+2j, 8t+2j+1) as
  * (rotl(P4, 4j) & 0x01E001E0) | (rotl(P2, T) & 0x82008200): sign at bit 15,
  * exponent field = e, mantissa = m/4, i.e. the code value times 2^-124
  * (e = 0 codes land on bf16 subnormals).

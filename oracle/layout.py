@@ -8,16 +8,17 @@ bit positions, no shared tables with the library.
 Layout definition (the library's packers must produce exactly this):
 
 * int8:  byte n*K + k  =  q[n, k] + 128  (offset binary).
-* int4:  byte n*K/2 + k//2 holds q[n, k] in bits 0..3 if k is even, 4..7 if odd.
+* int4:  little-endian 32-bit word t of row n (bytes n*K/2 + 4t ..) holds
+  k = 8t + 2r + h (r in 0..3, h in 0..1) in word bits 4r + 16h .. 4r + 16h + 3.
 * FP6 (2+4 split of each code c; sign = bit 5, e2 = bit 4, low piece = c & 0xF;
   the split into a 2-bit and a 4-bit piece follows the FP6-LLM / TC-FPx
   article, m.zhengruan.com news 124379, section "重新设计内核方案"):
     - bytes [0, N*K/4): 2-bit plane; bytes [N*K/4, 3*N*K/4): 4-bit plane.
     - 4-bit plane, little-endian 32-bit word t of row n at plane byte
-      n*K/2 + 4t, holds k = 8t + i, i = j + 4h (j in 0..3, h in 0..1); bit b of
-      the piece sits at word bit (5 + 16h - 4j + b) mod 32.
+      n*K/2 + 4t, holds k = 8t + 2j + h (j in 0..3, h in 0..1); bit b of the
+      piece sits at word bit (5 + 16h - 4j + b) mod 32.
     - 2-bit plane, little-endian 32-bit word u of row n at plane byte
-      n*K/4 + 4u, holds k = 16u + i, i = 8c + j + 4h; with
+      n*K/4 + 4u, holds k = 16u + 8c + 2j + h; with
       T = (0, 1, 4, 5, 8, 9, 12, 13)[4c + j] the sign bit sits at word bit
       (15 + 16h - T) mod 32 and e2 at (9 + 16h - T) mod 32.
 * bf16: the plain row-major bf16 matrix (no packing).
@@ -49,10 +50,11 @@ def unpack_int4(packed, N, K):
     assert b.size == N * K // 2
     q = np.empty((N, K), dtype=np.uint8)
     for n in range(N):
-        row = b[n * K // 2:(n + 1) * K // 2]
         for k in range(K):
-            byte = int(row[k // 2])
-            q[n, k] = (byte >> (4 * (k % 2))) & 0xF
+            t, i = divmod(k, 8)
+            r, h = i // 2, i % 2
+            w = _word(b, n * K // 2 + 4 * t)
+            q[n, k] = (w >> (4 * r + 16 * h)) & 0xF
     return q
 
 
@@ -75,7 +77,7 @@ def unpack_fp6(packed, N, K):
         for k in range(K):
             # 4-bit piece
             t, i = divmod(k, 8)
-            j, h = i % 4, i // 4
+            j, h = i // 2, i % 2
             w4 = _word(p4, n * K // 2 + 4 * t)
             four = 0
             for bb in range(4):
@@ -83,7 +85,7 @@ def unpack_fp6(packed, N, K):
             # 2-bit piece
             u, i16 = divmod(k, 16)
             c, rest = divmod(i16, 8)
-            j2, h2 = rest % 4, rest // 4
+            j2, h2 = rest // 2, rest % 2
             T = _T[4 * c + j2]
             w2 = _word(p2, n * K // 4 + 4 * u)
             sign = _bit(w2, 15 + 16 * h2 - T)

@@ -214,10 +214,11 @@ def test_fp6_layout_hand_examples(golden_dir):
 
 
 def test_int4_int8_layout_hand_examples():
-    # int4: k = 0 -> low nibble, k = 1 -> high nibble of byte 0
-    buf = bytes([0x21, 0x0F] + [0] * 30)
+    # int4 word 0 = 0x00F20301: k = 0 (bits 0..3) = 1, k = 1 (bits 16..19) = 2,
+    # k = 2 (bits 4..7) = 0, k = 3 (bits 20..23) = 15, k = 4 (bits 8..11) = 3
+    buf = bytes([0x01, 0x03, 0xF2, 0x00] + [0] * 28)
     q = layout.unpack_int4(buf, 1, 64)
-    assert q[0, :4].tolist() == [1, 2, 15, 0]
+    assert q[0, :6].tolist() == [1, 2, 0, 15, 3, 0]
     # int8 offset binary: 0x80 -> 0, 0x00 -> -128 (never produced), 0xFF -> 127, 0x01 -> -127
     q8 = layout.unpack_int8(bytes([0x80, 0xFF, 0x01] + [0x80] * 61), 1, 64)
     assert q8[0, :3].tolist() == [0, 127, -127]
