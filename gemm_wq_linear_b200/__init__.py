@@ -22,6 +22,8 @@ LIB_PATH = os.path.join(_HERE, "libwq.so")
 WQ_INT8, WQ_INT4, WQ_FP6_E3M2, WQ_BF16 = 0, 1, 2, 3
 FMT = {"int8": WQ_INT8, "int4": WQ_INT4, "fp6": WQ_FP6_E3M2, "bf16": WQ_BF16}
 WQ_LAUNCH_PDL = 0x1
+WQ_LAUNCH_TENSOR_CORES = 0x2
+WQ_LAUNCH_CUDA_CORES = 0x4
 STATUS = {0: "WQ_OK", 1: "WQ_ERR_NULL", 2: "WQ_ERR_SHAPE", 3: "WQ_ERR_FMT", 4: "WQ_ERR_GROUP",
           5: "WQ_ERR_ALIGN", 6: "WQ_ERR_CUDA", 7: "WQ_ERR_RANGE", 8: "WQ_ERR_TIMEOUT"}
 

@@ -174,7 +174,10 @@ wq_status wq_linear_ex(const void* x, const void* packed, const void* scales, co
   static const char* fn = "wq_linear";
   wq_status st = check_shape(fn, M, N, K, fmt, groupsize);
   if (st != WQ_OK) return st;
-  if (flags & ~WQ_LAUNCH_PDL) return set_error(WQ_ERR_SHAPE, "%s: unknown flags 0x%x", fn, flags);
+  if (flags & ~(WQ_LAUNCH_PDL | WQ_LAUNCH_TENSOR_CORES | WQ_LAUNCH_CUDA_CORES))
+    return set_error(WQ_ERR_SHAPE, "%s: unknown flags 0x%x", fn, flags);
+  if ((flags & WQ_LAUNCH_TENSOR_CORES) && (flags & WQ_LAUNCH_CUDA_CORES))
+    return set_error(WQ_ERR_SHAPE, "%s: flags select both kernels", fn);
   if (M == 0 || N == 0) return ok();
   if (!y) return set_error(WQ_ERR_NULL, "%s: y must be non-null", fn);
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
@@ -194,7 +197,14 @@ wq_status wq_linear_ex(const void* x, const void* packed, const void* scales, co
     return set_error(WQ_ERR_ALIGN, "%s: device pointers must be 16-byte aligned", fn);
   const int sms = sm_count_of_current_device();
   const int pdl = (flags & WQ_LAUNCH_PDL) ? 1 : 0;
-  if (M <= kGemvMaxM) {
+  bool gemv = M <= kGemvMaxM;
+  if (flags & WQ_LAUNCH_TENSOR_CORES) gemv = false;
+  if (flags & WQ_LAUNCH_CUDA_CORES) {
+    if (M > kGemvMaxM)
+      return set_error(WQ_ERR_SHAPE, "%s: the CUDA-core kernel takes M <= %d", fn, kGemvMaxM);
+    gemv = true;
+  }
+  if (gemv) {
     GemvParams p{};
     p.x = static_cast<const uint16_t*>(x);
     p.packed = packed;

@@ -42,9 +42,10 @@ namespace gemm {
 
 constexpr int kBM = 128;   // weight rows per tile (MMA M)
 constexpr int kBK = 128;   // k per pipeline stage
-constexpr int kThreads = 192;
-constexpr int kATileBytes = kBM * kBK * 2;  // 32 KB: two 64-column swizzle atoms
-constexpr int kNumA = 2;
+constexpr int kDqWarps = 16;                 // dequant / epilogue warps: 4 per TMEM lane quadrant
+constexpr int kThreads = 32 * (2 + kDqWarps);  // + producer warp + MMA warp
+constexpr int kACols = kBK / 2;  // TMEM columns of one A tile (two bf16 per column)
+constexpr int kXsSlots = 8;      // int4: ring of per-block group sums of x
 
 template <int FMT>
 struct Fmt;
@@ -69,10 +70,14 @@ template <int FMT, int MPAD>
 struct Layout {
   static constexpr int kXBytes = MPAD * 256;                    // two atoms of MPAD x 128 B
   static constexpr int kStage = Fmt<FMT>::kWBytes + kXBytes;   // multiple of 1024
-  static constexpr int kNumW = (FMT == WQ_BF16) ? 5 : ((FMT == WQ_INT4) ? 6 : 4);
+  // dequantized A tiles live in tensor memory (4 x 64 columns); shared memory
+  // holds only the packed-weight / activation ring, ~200 KB of it in flight
+  static constexpr int kNumA = 4;
+  static constexpr int kNumW0 = (200 * 1024) / kStage;
+  static constexpr int kNumW = kNumW0 > 16 ? 16 : kNumW0;
   static constexpr int kRingBytes = kNumW * kStage;
-  static constexpr int kABytes = (FMT == WQ_BF16) ? 0 : kNumA * kATileBytes;
   static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(kNumW >= 3, "too few stages");
 };
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
@@ -87,81 +92,51 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   else return r * 128 + 16 * (c ^ (r & 7));
 }
 
-// Store 8 bf16 (one 16-byte chunk, k = 8 ac .. 8 ac + 7 within a 64-column atom)
-// of row r into the A tile.
-__device__ __forceinline__ void st_a_chunk(uint8_t* A, int r, int k0, uint4 v) {
-  const int atom = k0 >> 6;
-  const int ac = (k0 & 63) >> 3;
-  *reinterpret_cast<uint4*>(A + atom * (kBM * 128) + swz<128>(r, ac)) = v;
-}
-
-// Decode row r of the packed stage tile into bf16 code values in A.
+// Decode the k-quarter u (32 k) of row r of the packed stage tile into 16 bf16
+// pairs (k, k + 1) of exact code values.
 template <int FMT>
-__device__ __forceinline__ void dequant_row(const uint8_t* W, uint8_t* A, int r) {
+__device__ __forceinline__ void dequant_quarter(const uint8_t* W, int r, int u, uint32_t (&p)[16]) {
   if constexpr (FMT == WQ_INT4) {
+    const uint4 w = *reinterpret_cast<const uint4*>(W + swz<64>(r, u));  // 16 B = 32 codes
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 w = *reinterpret_cast<const uint4*>(W + swz<64>(r, c));
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    for (int t = 0; t < 4; ++t) {
+      uint32_t q[4];
+      decode_int4_word(ws[t], q);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        uint32_t p[4];
-        decode_int4_word(ws[t], p);
-        st_a_chunk(A, r, 32 * c + 8 * t, make_uint4(p[0], p[1], p[2], p[3]));
-      }
+      for (int i = 0; i < 4; ++i) p[4 * t + i] = q[i];
     }
   } else if constexpr (FMT == WQ_FP6_E3M2) {
-    const uint8_t* W2 = W + kBM * 64;
-    uint32_t p4[16], p2[8];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 w = *reinterpret_cast<const uint4*>(W + swz<64>(r, c));
-      p4[4 * c + 0] = w.x;
-      p4[4 * c + 1] = w.y;
-      p4[4 * c + 2] = w.z;
-      p4[4 * c + 3] = w.w;
-    }
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const uint4 w = *reinterpret_cast<const uint4*>(W2 + swz<32>(r, c));
-      p2[4 * c + 0] = w.x;
-      p2[4 * c + 1] = w.y;
-      p2[4 * c + 2] = w.z;
-      p2[4 * c + 3] = w.w;
-    }
+    const uint4 w4 = *reinterpret_cast<const uint4*>(W + swz<64>(r, u));                  // 32 4-bit pieces
+    const uint2 w2 = *reinterpret_cast<const uint2*>(W + kBM * 64 + swz<32>(r, u >> 1) + 8 * (u & 1));  // 32 2-bit pieces
+    const uint32_t p4[4] = {w4.x, w4.y, w4.z, w4.w};
+    const uint32_t p2[2] = {w2.x, w2.y};
     constexpr uint32_t kRebias = 0x7D807D80u;  // bf16 2^124 in both halves
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      uint32_t p[8];
-      decode_fp6_words(p2[v], p4[2 * v], p4[2 * v + 1], p);
+    for (int v = 0; v < 2; ++v) {
+      uint32_t q[8];
+      decode_fp6_words(p2[v], p4[2 * v], p4[2 * v + 1], q);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        // value * 2^-124 (subnormal for e = 0) -> exact normal bf16 value
-        asm("mul.rn.bf16x2 %0, %0, %1;" : "+r"(p[j]) : "r"(kRebias));
+        asm("mul.rn.bf16x2 %0, %0, %1;" : "+r"(q[j]) : "r"(kRebias));  // exact normal values
+        p[8 * v + j] = q[j];
       }
-      st_a_chunk(A, r, 16 * v, make_uint4(p[0], p[1], p[2], p[3]));
-      st_a_chunk(A, r, 16 * v + 8, make_uint4(p[4], p[5], p[6], p[7]));
     }
   } else if constexpr (FMT == WQ_INT8) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 w = *reinterpret_cast<const uint4*>(W + swz<128>(r, c));
+    for (int c = 0; c < 2; ++c) {
+      const uint4 w = *reinterpret_cast<const uint4*>(W + swz<128>(r, 2 * u + c));
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-      uint32_t q[8];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         float f[4];
         decode_int8_word(ws[t], f);
-        q[2 * t] = pack_bf16x2_rn(f[0], f[1]);
-        q[2 * t + 1] = pack_bf16x2_rn(f[2], f[3]);
+        p[8 * c + 2 * t] = pack_bf16x2_rn(f[0], f[1]);
+        p[8 * c + 2 * t + 1] = pack_bf16x2_rn(f[2], f[3]);
       }
-      st_a_chunk(A, r, 16 * c, make_uint4(q[0], q[1], q[2], q[3]));
-      st_a_chunk(A, r, 16 * c + 8, make_uint4(q[4], q[5], q[6], q[7]));
     }
   }
 }
-
-__device__ __forceinline__ void dq_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -185,27 +160,33 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
   return v;
 }
 
-template <int FMT, int MPAD>
+// MPAD: MMA N (activation rows padded to a multiple of 8); MV <= MPAD: rows the
+// epilogue carries (the valid rows rounded up to a power of two).
+template <int FMT, int MPAD, int MV>
 __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_constant__ GemmParams a) {
   using L = Layout<FMT, MPAD>;
   constexpr int NW = L::kNumW;
+  constexpr int NA = L::kNumA;
   constexpr bool kInt4 = FMT == WQ_INT4;
+  constexpr bool kTmemA = FMT != WQ_BF16;  // bf16 weights are the A operand in shared memory as loaded
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment of the tiles (swizzle atoms and descriptors need it)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint8_t* atile = ring + L::kRingBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(atile + L::kABytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + L::kRingBytes);
   uint64_t* full_w = bars;             // [NW]  tensor copies landed
   uint64_t* empty_w = full_w + NW;     // [NW]  MMA finished with the stage
-  uint64_t* afull = empty_w + NW;      // [2]   A tile written
-  uint64_t* aempty = afull + kNumA;    // [2]   MMA finished with the A tile
-  uint64_t* dfull = aempty + kNumA;    // [8]   accumulator buffer complete
-  uint64_t* dempty = dfull + 8;        // [8]   accumulator buffer drained
-  uint64_t* done = dempty + 8;         // [1]   every MMA of the CTA completed
+  uint64_t* afull = empty_w + NW;      // [NA]  A tile written to TMEM
+  uint64_t* aempty = afull + NA;       // [NA]  MMA finished with the A tile
+  uint64_t* dfull = aempty + NA;       // [4]   accumulator (block-)buffer complete
+  uint64_t* dempty = dfull + 4;        // [4]   int4: accumulator block-buffer drained
+  uint64_t* xready = dempty + 4;       // [kXsSlots] int4: group sums of x of a block written
+  uint64_t* done = xready + kXsSlots;  // [1]   every MMA of the CTA completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   int* issued_slot = reinterpret_cast<int*>(tmem_slot + 1);
-  float* xsum = reinterpret_cast<float*>(tmem_slot + 4);  // int4: [groups][MPAD]
+  float* xs = reinterpret_cast<float*>(tmem_slot + 4);  // int4: [kXsSlots][4 groups][MV] group sums of x
+  // writer warps of the group sums: entries (activation row, 8-k chunk) = MV x 16
+  constexpr int kXsWarps = (MV * 16 + 31) / 32;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -217,11 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   const int kb0 = split * a.kb_per_split;
   const int nkb = max(0, min(a.kb_per_split, KB - kb0));
   const int g = kInt4 ? a.groupsize : kBK;
-  const int gpb = kBK / g;                                  // groups per k-block (int4)
-  const int kbeg = kb0 * kBK;
-  const int kend = min(a.K, (kb0 + nkb) * kBK);
-  const int ngroups = kInt4 ? (kend - kbeg) / g : 0;      // groups of this CTA
-  const int nd = kInt4 ? 2 * gpb : 1;                      // accumulator buffers
+  const int gpb = kBK / g;  // groups per k-block (int4)
+  // TMEM columns: [0, NA * 64) A tiles, then accumulators
+  constexpr uint32_t kDCol = NA * kACols;
+  const int ndb = kInt4 ? (gpb * MPAD <= 64 ? 4 : 2) : 1;  // int4 accumulator block-buffers
   const uint32_t tmem_cols = a.tmem_cols;
 
   if (a.pdl) pdl_launch_dependents();
@@ -230,14 +210,15 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
       mbar_init(&full_w[i], 1);
       mbar_init(&empty_w[i], 1);
     }
-    for (int i = 0; i < kNumA; ++i) {
-      mbar_init(&afull[i], 4);
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(&afull[i], kDqWarps);
       mbar_init(&aempty[i], 1);
     }
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&dfull[i], 1);
       mbar_init(&dempty[i], 4);
     }
+    for (int i = 0; i < kXsSlots; ++i) mbar_init(&xready[i], kXsWarps);
     mbar_init(done, 1);
     *issued_slot = 0;
     fence_mbar_init();
@@ -249,9 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   const uint32_t tmem = *tmem_slot;
 
   bool failed = false;
-  float acc[MPAD];
+  float acc[MV];
 #pragma unroll
-  for (int m = 0; m < MPAD; ++m) acc[m] = 0.f;
+  for (int m = 0; m < MV; ++m) acc[m] = 0.f;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -302,44 +283,43 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, MPAD);
-      int dcount = 0;  // int4: accumulator buffers used so far
       for (int j = 0; j < nkb && !failed; ++j) {
         const int s = j % NW;
-        const int ai = j % kNumA;
-        uint8_t* A;
-        if constexpr (FMT == WQ_BF16) {
-          if (!mbar_wait(&full_w[s], (j / NW) & 1)) { failed = true; break; }
-          A = ring + size_t(s) * L::kStage;
-        } else {
-          if (!mbar_wait(&afull[ai], (j / kNumA) & 1)) { failed = true; break; }
-          A = atile + size_t(ai) * kATileBytes;
+        const int ai = j % NA;
+        if (!mbar_wait(kTmemA ? &afull[ai] : &full_w[s], kTmemA ? ((j / NA) & 1) : ((j / NW) & 1))) {
+          failed = true;
+          break;
         }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(A);
         const uint32_t b_base = smem_u32(ring + size_t(s) * L::kStage + Fmt<FMT>::kWBytes);
-        if constexpr (kInt4) {
-          const int kvalid = min(kBK, a.K - (kb0 + j) * kBK);
-          for (int gi = 0; gi < gpb && gi * g < kvalid; ++gi, ++dcount) {
-            const int b = dcount % nd;
-            if (!mbar_wait(&dempty[b], ((dcount / nd) & 1) ^ 1)) { failed = true; break; }
-            tc_fence_after();
-            for (int kk = gi * (g / 16); kk < (gi + 1) * (g / 16); ++kk) {
-              const uint32_t ao = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-              const uint32_t bo = (kk >> 2) * (MPAD * 128) + (kk & 3) * 32;
-              mma_bf16(tmem + b * MPAD, smem_desc_sw128(a_base + ao), smem_desc_sw128(b_base + bo), idesc,
-                       kk != gi * (g / 16));
-            }
-            mma_commit(&dfull[b]);
+        const uint32_t a_tm = tmem + ai * kACols;
+        const uint32_t a_sm = smem_u32(ring + size_t(s) * L::kStage);
+        auto mma_step = [&](uint32_t d, int kk, bool accum) {
+          const uint64_t bd = smem_desc_sw128(b_base + (kk >> 2) * (MPAD * 128) + (kk & 3) * 32);
+          if constexpr (kTmemA) {
+            mma_bf16_tmem_a(d, a_tm + kk * 8, bd, idesc, accum);
+          } else {
+            mma_bf16(d, smem_desc_sw128(a_sm + (kk >> 2) * (kBM * 128) + (kk & 3) * 32), bd, idesc, accum);
           }
+        };
+        if constexpr (kInt4) {
+          // every group of the block into its own MPAD-column accumulator
+          const int db = j & (ndb - 1);
+          if (!mbar_wait(&dempty[db], ((j / ndb) & 1) ^ 1)) {
+            failed = true;
+            break;
+          }
+          tc_fence_after();
+          const int kvalid = min(kBK, a.K - (kb0 + j) * kBK);
+          for (int gi = 0; gi < gpb && gi * g < kvalid; ++gi)
+            for (int kk = gi * (g / 16); kk < (gi + 1) * (g / 16); ++kk)
+              mma_step(tmem + kDCol + (db * gpb + gi) * MPAD, kk, kk != gi * (g / 16));
+          mma_commit(&dfull[db]);
         } else {
 #pragma unroll 1
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint32_t ao = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-            const uint32_t bo = (kk >> 2) * (MPAD * 128) + (kk & 3) * 32;
-            mma_bf16(tmem, smem_desc_sw128(a_base + ao), smem_desc_sw128(b_base + bo), idesc, (j | kk) != 0);
-          }
+          for (int kk = 0; kk < kBK / 16; ++kk) mma_step(tmem + kDCol, kk, (j | kk) != 0);
         }
-        if constexpr (FMT != WQ_BF16) mma_commit(&aempty[ai]);
+        if constexpr (kTmemA) mma_commit(&aempty[ai]);  // A tile free
         mma_commit(&empty_w[s]);
       }
       if (!kInt4) mma_commit(&dfull[0]);  // accumulator complete
@@ -348,84 +328,118 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------------------ dequant + epilogue
-    const int r = 32 * (warp & 3) + lane;  // TMEM lane quadrant of this warp
+    // warp 2 + d: TMEM lane quadrant q = warp % 4 (rows 32 q ..), k-quarter u = d / 4
+    const int d = warp - 2;
+    const int u = d >> 2;
+    const int r = 32 * (warp & 3) + lane;
     const int n = n0 + r;
-    const uint32_t taddr_row = tmem + (uint32_t(32 * (warp & 3)) << 16);
+    const int dtid = threadIdx.x - 64;  // 0 .. 511 (warp d holds entries 32 d ..)
+    const uint32_t trow = uint32_t(32 * (warp & 3)) << 16;  // TMEM lane base of this warp
+    const int G = kInt4 ? a.K / g : 0;
     if (a.pdl) pdl_wait();
-    if constexpr (kInt4) {
-      // sums of x over every group of this CTA's k range
-      for (int idx = threadIdx.x - 64; idx < ngroups * MPAD; idx += 128) {
-        const int gl = idx / MPAD;
-        const int m = idx - gl * MPAD;
-        float sacc = 0.f;
-        if (m < a.M) {
-          const uint4* xp = reinterpret_cast<const uint4*>(a.x + size_t(m) * a.K + kbeg + gl * g);
-          for (int q = 0; q < g / 8; ++q) {
-            const uint4 v = __ldg(xp + q);
-            sacc += (bf16_lo_f(v.x) + bf16_hi_f(v.x)) + (bf16_lo_f(v.y) + bf16_hi_f(v.y)) +
-                    (bf16_lo_f(v.z) + bf16_hi_f(v.z)) + (bf16_lo_f(v.w) + bf16_hi_f(v.w));
-          }
-        }
-        xsum[idx] = sacc;
-      }
-      dq_sync();
-    }
-    int gdone = 0;  // int4: groups folded into acc so far
-    // int4: fold the accumulator buffers of groups [gdone, upto) into acc
-    auto fold_groups = [&](int upto) {
+    // int4: scale and zero of this row for the groups of the block this warp folds
+    float sz_s[4], sz_z[4];
+    auto load_sz = [&](int j) {
       if constexpr (kInt4) {
-        const int G = a.K / g;
-        for (; gdone < upto && !failed; ++gdone) {
-          const int b = gdone % nd;
-          if (!mbar_wait(&dfull[b], (gdone / nd) & 1)) { failed = true; break; }
-          tc_fence_after();
-          uint32_t d[MPAD];
-          tmem_ld_32x32b<MPAD>(taddr_row + b * MPAD, d);
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&dempty[b]);
-          if (n < a.N) {
-            const size_t gi = size_t(n) * G + (kbeg / g) + gdone;
-            const float sc = bf16f(a.scales[gi]);
-            const float zc = fmaf(-128.f, sc, bf16f(a.zeros[gi]));
-            const float* xs = xsum + gdone * MPAD;
+        const int gbase = (kb0 + j) * (kBK / g);
 #pragma unroll
-            for (int m = 0; m < MPAD; ++m) acc[m] = fmaf(sc, __uint_as_float(d[m]), fmaf(zc, xs[m], acc[m]));
-          }
+        for (int gi = 0; gi < 4; ++gi) {
+          const bool ok = gi < gpb && n < a.N && (kb0 + j) * kBK + gi * g < a.K;
+          const size_t gidx = size_t(n) * G + gbase + gi;
+          sz_s[gi] = ok ? bf16f(a.scales[gidx]) : 0.f;
+          sz_z[gi] = ok ? bf16f(a.zeros[gidx]) : 0.f;
         }
       }
     };
-    if constexpr (FMT != WQ_BF16) {
+    // int4: fold the group accumulators of block j into acc (warps with u == j % 4)
+    auto fold_block = [&](int j) {
+      if constexpr (kInt4) {
+        const int db = j & (ndb - 1);
+        if (!mbar_wait(&dfull[db], (j / ndb) & 1) || !mbar_wait(&xready[j % kXsSlots], (j / kXsSlots) & 1)) {
+          failed = true;
+          return;
+        }
+        tc_fence_after();
+        const int kvalid = min(kBK, a.K - (kb0 + j) * kBK);
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) {
+          if (gi < gpb && gi * g < kvalid) {
+            constexpr int LD = MV <= 8 ? 8 : MV;  // columns loaded per group
+            uint32_t dv[LD];
+            tmem_ld_32x32b<LD>(tmem + trow + kDCol + (db * gpb + gi) * MPAD, dv);
+            tmem_ld_wait();
+            const float sc = sz_s[gi];
+            const float zc = fmaf(-128.f, sc, sz_z[gi]);
+            const float* xg = xs + ((j % kXsSlots) * 4 + gi) * MV;
+#pragma unroll
+            for (int m = 0; m < MV; ++m) acc[m] = fmaf(sc, __uint_as_float(dv[m]), fmaf(zc, xg[m], acc[m]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dempty[db]);
+      }
+    };
+    if constexpr (kTmemA) {
       for (int j = 0; j < nkb && !failed; ++j) {
         const int s = j % NW;
-        const int ai = j % kNumA;
+        const int ai = j % NA;
+        if (kInt4 && (j & 3) == u) load_sz(j);
         if (!mbar_wait(&full_w[s], (j / NW) & 1)) { failed = true; break; }
-        if (!mbar_wait(&aempty[ai], ((j / kNumA) & 1) ^ 1)) { failed = true; break; }
-        dequant_row<FMT>(ring + size_t(s) * L::kStage, atile + size_t(ai) * kATileBytes, r);
-        fence_proxy_async_smem();
+        const uint8_t* st = ring + size_t(s) * L::kStage;
+        uint32_t pv[16];
+        dequant_quarter<FMT>(st, r, u, pv);
+        if (!mbar_wait(&aempty[ai], ((j / NA) & 1) ^ 1)) { failed = true; break; }
+        tc_fence_after();
+        tmem_st_32x32b_x16(tmem + trow + ai * kACols + 16 * u, pv);
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&afull[ai]);
-        // fold the groups of the previous k-block while the MMA runs on this one
-        if constexpr (kInt4) fold_groups(min(ngroups, j * gpb));
+        if constexpr (kInt4) {
+          // group sums of x for this block from the B tile (the first kXsWarps
+          // warps; entry e = 16 m + c, chunk c of 8 k), then fold block j - 1
+          if (d < kXsWarps) {
+            const uint8_t* xt = st + Fmt<FMT>::kWBytes;
+            const int e = dtid;
+            const int m = e >> 4;
+            const int c = e & 15;
+            float sacc = 0.f;
+            if (m < MV) {
+              const uint4 v = *reinterpret_cast<const uint4*>(xt + (c >> 3) * (MPAD * 128) + swz<128>(m, c & 7));
+              sacc = (bf16_lo_f(v.x) + bf16_hi_f(v.x)) + (bf16_lo_f(v.y) + bf16_hi_f(v.y)) +
+                     (bf16_lo_f(v.z) + bf16_hi_f(v.z)) + (bf16_lo_f(v.w) + bf16_hi_f(v.w));
+            }
+            // the g / 8 chunks of a group sit in consecutive, aligned lanes
+            for (int o = 1; o < g / 8; o <<= 1) sacc += __shfl_xor_sync(0xFFFFFFFFu, sacc, o);
+            if (m < MV && (c & (g / 8 - 1)) == 0) xs[((j % kXsSlots) * 4 + c / (g / 8)) * MV + m] = sacc;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xready[j % kXsSlots]);
+          }
+          if (j >= 1 && ((j - 1) & 3) == u) fold_block(j - 1);
+        }
+      }
+      if constexpr (kInt4) {
+        if (!failed && nkb >= 1 && ((nkb - 1) & 3) == u) fold_block(nkb - 1);
       }
     }
-    if constexpr (kInt4) {
-      fold_groups(ngroups);
-    } else if (!failed) {
-      if (mbar_wait(&dfull[0], 0)) {
-        tc_fence_after();
-        uint32_t d[MPAD];
-        tmem_ld_32x32b<MPAD>(taddr_row, d);
-        tmem_ld_wait();
-        float sc = 1.f;
-        if (n < a.N) {
-          if constexpr (FMT == WQ_INT8 || FMT == WQ_FP6_E3M2) sc = fp16f(a.scales[n]);
-        }
+    if constexpr (!kInt4) {
+      if (!failed && u == 0) {
+        if (mbar_wait(&dfull[0], 0)) {
+          tc_fence_after();
+          constexpr int LD = MV <= 8 ? 8 : MV;
+          uint32_t dv[LD];
+          tmem_ld_32x32b<LD>(tmem + trow + kDCol, dv);
+          tmem_ld_wait();
+          float sc = 1.f;
+          if (n < a.N) {
+            if constexpr (FMT == WQ_INT8 || FMT == WQ_FP6_E3M2) sc = fp16f(a.scales[n]);
+          }
 #pragma unroll
-        for (int m = 0; m < MPAD; ++m) acc[m] = __uint_as_float(d[m]) * sc;
-      } else {
-        failed = true;
+          for (int m = 0; m < MV; ++m) acc[m] = __uint_as_float(dv[m]) * sc;
+        } else {
+          failed = true;
+        }
       }
     }
   }
@@ -446,39 +460,60 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   if (warp == 1) tmem_dealloc(tmem, tmem_cols);
 
   const bool epi = warp >= 2;
+  const int u = (warp - 2) >> 2;
   const int r = 32 * (warp & 3) + lane;
   const int n = n0 + r;
-  if (S == 1) {
-    if (epi && !any_failed && n < a.N) {
+  // int4: the four k-quarter warp groups each folded a quarter of the blocks;
+  // partials meet in the (now idle) ring
+  float* red = reinterpret_cast<float*>(ring);  // [3][128][MV]
+  if (kInt4) {
+    if (epi && u > 0) {
 #pragma unroll
-      for (int m = 0; m < MPAD; ++m)
+      for (int m = 0; m < MV; ++m) red[((u - 1) * 128 + r) * MV + m] = acc[m];
+    }
+    __syncthreads();
+    if (epi && u == 0) {
+#pragma unroll
+      for (int q = 0; q < 3; ++q)
+#pragma unroll
+        for (int m = 0; m < MV; ++m) acc[m] += red[(q * 128 + r) * MV + m];
+    }
+  }
+  const bool out = epi && u == 0;
+  if (S == 1) {
+    if (out && !any_failed && n < a.N) {
+#pragma unroll
+      for (int m = 0; m < MV; ++m)
         if (m < a.M) a.y[size_t(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[m]));
     }
     return;
   }
   // split-K over the cluster: partials through distributed shared memory
-  float* red = reinterpret_cast<float*>(ring);  // [128][MPAD], the ring is idle now
-  if (epi) {
+  constexpr int MV4 = MV < 4 ? 4 : MV;                          // row pitch of the partial buffer (16-byte units)
+  float* part = reinterpret_cast<float*>(ring) + 3 * 128 * MV;  // [128][MV4], after the int4 partials
+  if (out) {
 #pragma unroll
-    for (int m = 0; m < MPAD; m += 4)
-      *reinterpret_cast<float4*>(red + r * MPAD + m) = make_float4(acc[m], acc[m + 1], acc[m + 2], acc[m + 3]);
+    for (int m = 0; m < MV4; m += 4)
+      *reinterpret_cast<float4*>(part + r * MV4 + m) =
+          make_float4(m < MV ? acc[m] : 0.f, m + 1 < MV ? acc[m + 1] : 0.f, m + 2 < MV ? acc[m + 2] : 0.f,
+                      m + 3 < MV ? acc[m + 3] : 0.f);
   }
   cluster_sync_all();
-  if (cluster_ctarank() == 0 && epi && !any_failed && n < a.N) {
-    const uint32_t base = smem_u32(red + r * MPAD);
+  if (cluster_ctarank() == 0 && out && !any_failed && n < a.N) {
+    const uint32_t base = smem_u32(part + r * MV4);
     for (int q = 1; q < S; ++q) {
       const uint32_t rb = map_to_rank(base, uint32_t(q));
 #pragma unroll
-      for (int m = 0; m < MPAD; m += 4) {
+      for (int m = 0; m < MV4; m += 4) {
         const float4 v = ld_cluster_f4(rb + m * 4);
-        acc[m] += v.x;
-        acc[m + 1] += v.y;
-        acc[m + 2] += v.z;
-        acc[m + 3] += v.w;
+        if (m < MV) acc[m] += v.x;
+        if (m + 1 < MV) acc[m + 1] += v.y;
+        if (m + 2 < MV) acc[m + 2] += v.z;
+        if (m + 3 < MV) acc[m + 3] += v.w;
       }
     }
 #pragma unroll
-    for (int m = 0; m < MPAD; ++m)
+    for (int m = 0; m < MV; ++m)
       if (m < a.M) a.y[size_t(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[m]));
   }
   cluster_sync_all();  // keep every CTA's shared memory alive until rank 0 has read it
@@ -487,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
 }  // namespace gemm
 
 // ----------------------------------------------------------------- launcher
-template <int FMT, int MPAD>
+template <int FMT, int MPAD, int MV>
 static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int sm_count) {
   using L = gemm::Layout<FMT, MPAD>;
   GemmParams p = p0;
@@ -496,22 +531,18 @@ static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int 
   // split K over a cluster so that about one CTA per SM is busy; int4 keeps each
   // CTA's k range at most 4096 (the per-group x sums live in shared memory)
   int S = (sm_count + tiles / 2) / tiles;
-  if (FMT == WQ_INT4) S = S < (p.K + 4095) / 4096 ? (p.K + 4095) / 4096 : S;
   if (S > 8) S = 8;
   if (S > KB) S = KB;
   if (S < 1) S = 1;
   int kbps = (KB + S - 1) / S;
   S = (KB + kbps - 1) / kbps;
-  if (FMT == WQ_INT4 && kbps * gemm::kBK > 4096) return cudaErrorInvalidValue;  // K > 32768 for int4
   p.splits = S;
   p.kb_per_split = kbps;
-  const int g = FMT == WQ_INT4 ? p.groupsize : gemm::kBK;
-  const int nd = FMT == WQ_INT4 ? 2 * (gemm::kBK / g) : 1;
-  uint32_t cols = 32;
-  while (cols < uint32_t(nd * MPAD)) cols <<= 1;
-  p.tmem_cols = cols;
-  const size_t xsum_bytes = FMT == WQ_INT4 ? size_t(kbps * gemm::kBK / g) * MPAD * 4 : 0;
-  const size_t smem = 1024 + L::kRingBytes + L::kABytes + 64 * 8 + 64 + xsum_bytes;
+  p.tmem_cols = 512;  // A tiles (4 x 64 columns) + accumulators (<= 256 columns)
+  const size_t small = 1024 + 64 * 8 + 64 + size_t(gemm::kXsSlots * 4 * MV) * 4;
+  const size_t smem = L::kRingBytes + small;
+  static_assert(L::kRingBytes >= (3 * 128 * MV + 128 * (MV < 4 ? 4 : MV)) * 4,
+                "reduction buffers must fit the idle ring");
 
   cudaError_t e;
   const uint8_t* w = static_cast<const uint8_t*>(p.packed);
@@ -528,10 +559,10 @@ static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int 
   }
   if (e == cudaSuccess) e = make_tmap_2d(&p.tm_x, p.x, 2, uint64_t(p.K), p.M, uint64_t(p.K) * 2, 64, MPAD, 128);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gemm::wq_gemm_kernel<FMT, MPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  e = cudaFuncSetAttribute(gemm::wq_gemm_kernel<FMT, MPAD, MV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   if (S > 1) {
-    e = cudaFuncSetAttribute(gemm::wq_gemm_kernel<FMT, MPAD>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(gemm::wq_gemm_kernel<FMT, MPAD, MV>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
@@ -555,14 +586,19 @@ static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int 
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemm::wq_gemm_kernel<FMT, MPAD>, p);
+  return cudaLaunchKernelEx(&cfg, gemm::wq_gemm_kernel<FMT, MPAD, MV>, p);
 }
 
+// The MMA's N (activation rows) is padded to 16 or 32 (a multiple of 16 is
+// required with A in tensor memory); the epilogue carries only MV rows.
 template <int FMT>
 static cudaError_t launch_gemm_fmt(const GemmParams& p, cudaStream_t s, int sms) {
-  if (p.M <= 8) return launch_gemm_t<FMT, 8>(p, s, sms);
-  if (p.M <= 16) return launch_gemm_t<FMT, 16>(p, s, sms);
-  return launch_gemm_t<FMT, 32>(p, s, sms);
+  if (p.M <= 1) return launch_gemm_t<FMT, 16, 1>(p, s, sms);
+  if (p.M <= 2) return launch_gemm_t<FMT, 16, 2>(p, s, sms);
+  if (p.M <= 4) return launch_gemm_t<FMT, 16, 4>(p, s, sms);
+  if (p.M <= 8) return launch_gemm_t<FMT, 16, 8>(p, s, sms);
+  if (p.M <= 16) return launch_gemm_t<FMT, 16, 16>(p, s, sms);
+  return launch_gemm_t<FMT, 32, 32>(p, s, sms);
 }
 
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t s, int sms) {

@@ -113,6 +113,15 @@ __device__ __forceinline__ void load_x_smem(XRegs<FMT, MM>& xr, const uint8_t* x
         xr.v[m][8 * q + 2 * i + 1] = bf16_hi_f(w[i]);
       }
     }
+    if constexpr (FMT == WQ_INT4) {
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < GemvFmt<FMT>::kLaneK; i += 2) {
+        s0 += xr.v[m][i];
+        s1 += xr.v[m][i + 1];
+      }
+      xr.xsum[m] = s0 + s1;
+    }
   }
 }
 
@@ -179,7 +188,6 @@ __device__ __forceinline__ void lane_dot(const uint8_t* w, const uint8_t* w2p, i
   for (int m = 0; m < MM; ++m) acc[m] = a0[m] + a1[m];
 }
 
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory"); }
 
 template <int FMT, int MM>
 __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kernel(const __grid_constant__ GemvParams a) {
@@ -197,9 +205,11 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
   const int C = (a.K + kChunkK - 1) / kChunkK;
   const int n0 = blockIdx.x * a.rows_per_cta;
   const int R = min(a.rows_per_cta, a.N - n0);
-  float* xsum_s = part + size_t(C) * a.rows_per_cta * MM;  // int4: [K/32][MM]
   const int NRB = (R + kRB - 1) / kRB;
   const int T = C * NRB;
+  // stages run chunk-major over the CTA's row blocks; each CTA starts at a
+  // different chunk so that concurrent CTAs fetch different parts of x
+  const int c_rot = blockIdx.x % C;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -226,7 +236,9 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
     }
     auto issue_x = [&](int t) {
       const int s = t % NS;
-      const int c = t / NRB;
+      if (t % NRB != 0) return;  // x of a chunk travels with the chunk's first stage only
+      int c = t / NRB + c_rot;
+      c = c >= C ? c - C : c;
       const int kc = min(kChunkK, a.K - c * kChunkK);
       if (lane < MM)
         bulk_g2s(ring + size_t(s) * L::kStageBytes + kRB * F::kRowBytes + lane * L::kXBytes,
@@ -239,13 +251,14 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
         failed = true;
         break;
       }
-      const int c = t / NRB;
-      const int rb = t - c * NRB;
+      const int ci = t / NRB;
+      const int rb = t - ci * NRB;
+      const int c = ci + c_rot >= C ? ci + c_rot - C : ci + c_rot;
       const int rows = min(kRB, R - rb * kRB);
       const int nbox = (rows + BH - 1) / BH;
       const int kc = min(kChunkK, a.K - c * kChunkK);
       if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], uint32_t(nbox * BH * F::kRowBytes) + MM * uint32_t(kc) * 2);
+        mbar_arrive_expect_tx(&full[s], uint32_t(nbox * BH * F::kRowBytes) + (rb == 0 ? MM * uint32_t(kc) * 2 : 0u));
         uint8_t* st = ring + size_t(s) * L::kStageBytes;
         for (int b = 0; b < nbox; ++b) {
           const int row = n0 + rb * kRB + b * BH;
@@ -273,24 +286,6 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
     const int cw = warp - 1;
     const int ctid = threadIdx.x - 32;
     if (a.pdl) pdl_wait();
-    if constexpr (FMT == WQ_INT4) {
-      // sum of x over every 32-k block of every activation row (for the zero fold)
-      const int nblk = a.K / 32;
-      for (int idx = ctid; idx < nblk * MM; idx += kConsumerWarps * 32) {
-        const int m = idx % MM;
-        const int blk = idx / MM;
-        const uint4* xp = reinterpret_cast<const uint4*>(a.x + size_t(m) * a.K + blk * 32);
-        float sacc = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 v = __ldg(xp + q);
-          sacc += (bf16_lo_f(v.x) + bf16_hi_f(v.x)) + (bf16_lo_f(v.y) + bf16_hi_f(v.y)) +
-                  (bf16_lo_f(v.z) + bf16_hi_f(v.z)) + (bf16_lo_f(v.w) + bf16_hi_f(v.w));
-        }
-        xsum_s[idx] = sacc;
-      }
-      consumer_sync();
-    }
     int cur_c = -1;
     XRegs<FMT, MM> xr;
     constexpr int J = kRB / kConsumerWarps;  // rows of a stage this warp takes (4)
@@ -301,8 +296,9 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
     auto fetch_sz = [&](int t, uint32_t* dst) {
       if constexpr (FMT == WQ_INT4) {
         if (t >= T) return;
-        const int c = t / NRB;
-        const int rb = t - c * NRB;
+        const int ci = t / NRB;
+        const int rb = t - ci * NRB;
+        const int c = ci + c_rot >= C ? ci + c_rot - C : ci + c_rot;
         const int rows = min(kRB, R - rb * kRB);
         const int k0 = c * kChunkK + lane * F::kLaneK;
         if (k0 >= a.K) return;
@@ -338,8 +334,9 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
         failed = true;
         break;
       }
-      const int c = t / NRB;
-      const int rb = t - c * NRB;
+      const int ci = t / NRB;
+      const int rb = t - ci * NRB;
+      const int c = ci + c_rot >= C ? ci + c_rot - C : ci + c_rot;
       const int rows = min(kRB, R - rb * kRB);
       const int k0 = c * kChunkK + lane * F::kLaneK;
       const bool active = k0 < a.K;
@@ -347,10 +344,6 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
       if (c != cur_c) {
         if (active) {
           load_x_smem<FMT, MM>(xr, st + kRB * F::kRowBytes, lane);
-          if constexpr (FMT == WQ_INT4) {
-#pragma unroll
-            for (int m = 0; m < MM; ++m) xr.xsum[m] = xsum_s[(k0 / 32) * MM + m];
-          }
         }
         cur_c = c;
       }
@@ -438,7 +431,6 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   using F = GemvFmt<FMT>;
   GemvParams p = p0;
   const int C = (p.K + L::kChunkK - 1) / L::kChunkK;
-  const size_t xsum_bytes = (FMT == WQ_INT4) ? size_t(p.K / 32) * MM * 4 : 0;
   const int target = sm_count * gemv_ctas_per_sm(MM);
   const size_t kGemvSmemBudget = kGemvSmemPerSm / gemv_ctas_per_sm(MM);
   // rows per CTA: a multiple of the box height, about N / target
@@ -449,13 +441,13 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   if (R < kBoxRows) R = kBoxRows;
   p.rows_per_cta = R;
   p.box_rows = kBoxRows;
-  const size_t fixed = 16 * 8 + 16 + size_t(C) * R * MM * 4 + xsum_bytes;
+  const size_t fixed = 16 * 8 + 16 + size_t(C) * R * MM * 4;
   if (fixed + 2 * size_t(L::kStageBytes) > 200 * 1024) return cudaErrorInvalidValue;
   int stages = fixed < kGemvSmemBudget ? int((kGemvSmemBudget - fixed) / L::kStageBytes) : 2;
   if (stages > 8) stages = 8;
   if (stages < 2) stages = 2;
   p.stages = stages;
-  const size_t smem = size_t(stages) * L::kStageBytes + size_t(stages) * 16 + 16 + size_t(C) * R * MM * 4 + xsum_bytes;
+  const size_t smem = size_t(stages) * L::kStageBytes + size_t(stages) * 16 + 16 + size_t(C) * R * MM * 4;
 
   // tensor maps: rows of packed bytes viewed as 32-bit elements, one chunk per box
   cudaError_t e;

@@ -158,6 +158,9 @@ wq_status wq_linear(const void* x, const void* packed, const void* scales, const
                               flight on the stream; x is read and y written only after
                               the previous kernel has completed. */
 
+#define WQ_LAUNCH_TENSOR_CORES 0x2u /* run the tcgen05 swap-AB kernel whatever M is */
+#define WQ_LAUNCH_CUDA_CORES 0x4u   /* run the CUDA-core GEMV (M <= 4 only) */
+
 /* wq_linear with launch-option flags (0 = exactly wq_linear). */
 wq_status wq_linear_ex(const void* x, const void* packed, const void* scales, const void* zeros,
                        void* y, int64_t M, int64_t N, int64_t K, int fmt, int groupsize,

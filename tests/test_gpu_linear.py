@@ -42,6 +42,26 @@ def test_linear_matches_oracle(fmt, g, M):
 
 
 @pytest.mark.parametrize("fmt,g", VARIANTS)
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+def test_linear_tensor_core_kernel_small_m(fmt, g, M):
+    """The tcgen05 kernel selected explicitly for the GEMV's range of M."""
+    Wd, pw = _case(fmt, g)
+    x = workloads.activations(M, K_SMALL, seed=2000 + M)
+    y = gpu_linear(x, pw, flags=wq.WQ_LAUNCH_TENSOR_CORES)
+    compare(y, linear.linear_ref(x_bits(x), Wd))
+
+
+@pytest.mark.parametrize("fmt,g", VARIANTS)
+@pytest.mark.parametrize("M", [1, 3, 4])
+def test_linear_cuda_core_kernel(fmt, g, M):
+    """The CUDA-core GEMV selected explicitly."""
+    Wd, pw = _case(fmt, g)
+    x = workloads.activations(M, K_SMALL, seed=3000 + M)
+    y = gpu_linear(x, pw, flags=wq.WQ_LAUNCH_CUDA_CORES)
+    compare(y, linear.linear_ref(x_bits(x), Wd))
+
+
+@pytest.mark.parametrize("fmt,g", VARIANTS)
 def test_linear_pdl_flag_same_result(fmt, g):
     Wd, pw = _case(fmt, g)
     x = workloads.activations(2, K_SMALL, seed=77).cuda()
