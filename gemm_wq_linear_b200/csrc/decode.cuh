@@ -1,10 +1,15 @@
 // In-register weight decode for the wq kernels (sm_100a).
 //
-// Each decoder turns packed 32-bit words into bf16 pairs (or fp32 values) with a
+// Each decoder turns packed 32-bit words into bf16 pairs or fp32 values with a
 // few bit operations, in the spirit of the SIMT bit-parallel dequantization of
 // the FP6-LLM / TC-FPx article (m.zhengruan.com news 124379, section
 // "重新设计内核方案": dequantize inside registers with bit-level parallelism and
 // splice the 2-bit and 4-bit pieces of each 6-bit weight in parallel).
+//
+// The bit operations are written as explicit PTX (lop3 with its truth table,
+// funnel shifts) so that every mask-and-merge is one LOP3 instruction: the
+// CUDA-core GEMV is bound by the integer ALU pipe, and its throughput is the
+// number of ALU instructions per weight.
 //
 // Pair convention: a decoded pair register holds (lo, hi) = (k, k + 1); the
 // packers place the codes inside each word so that this needs no permutation.
@@ -13,70 +18,48 @@
 
 namespace wq {
 
-// bf16 bit pattern of 128.0 in both halves: OR-ing a 4-bit code into the low
-// mantissa bits gives the exact value 128 + q.
-constexpr uint32_t kBf16Magic128x2 = 0x43004300u;
-
+// ------------------------------------------------------------------ primitives
+// (a & b) | c in one LOP3 (truth table 0xEA = (0xF0 & 0xCC) | 0xAA).
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// a & b in one LOP3.
+__device__ __forceinline__ uint32_t lop_and(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, 0, 0xC0;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 __device__ __forceinline__ uint32_t rotl32(uint32_t x, int s) { return __funnelshift_l(x, x, s); }
 
-// int4: word w holds q[8t + 2r + h] in bits 4r + 16h .. +3.  Output p[r] = bf16
-// pair (128 + q[8t + 2r], 128 + q[8t + 2r + 1]), r = 0..3.
-__device__ __forceinline__ void decode_int4_word(uint32_t w, uint32_t p[4]) {
-  p[0] = (w & 0x000F000Fu) | kBf16Magic128x2;
-  p[1] = ((w >> 4) & 0x000F000Fu) | kBf16Magic128x2;
-  p[2] = ((w >> 8) & 0x000F000Fu) | kBf16Magic128x2;
-  p[3] = ((w >> 12) & 0x000F000Fu) | kBf16Magic128x2;
+// (a0, a1) += (b0, b1): packed fp32 add of sm_100 (one instruction, two lanes).
+__device__ __forceinline__ void fadd2(float& a0, float& a1, float b0, float b1) {
+  asm("{.reg .b64 a, b;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "mov.b64 b, {%2, %3};\n\t"
+      "add.rn.f32x2 a, a, b;\n\t"
+      "mov.b64 {%0, %1}, a;}\n"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
 }
 
-// FP6 (2+4 planes): p2 is the 2-bit-plane word of 16 weights, p4a / p4b the two
-// 4-bit-plane words of its first and second 8 weights.  Output p[4c + j] = bf16
-// pair (k = 8c + 2j, 8c + 2j + 1) holding code value * 2^-124 (subnormal for e = 0).
-__device__ __forceinline__ void decode_fp6_words(uint32_t p2, uint32_t p4a, uint32_t p4b, uint32_t p[8]) {
-  constexpr uint32_t kFour = 0x01E001E0u;  // bits 5..8 of each half: (e1 e0 m1 m0)
-  constexpr uint32_t kTwo = 0x82008200u;   // bits 15 and 9 of each half: sign, e2
-  p[0] = (p4a & kFour) | (p2 & kTwo);
-  p[1] = (rotl32(p4a, 4) & kFour) | (rotl32(p2, 1) & kTwo);
-  p[2] = (rotl32(p4a, 8) & kFour) | (rotl32(p2, 4) & kTwo);
-  p[3] = (rotl32(p4a, 12) & kFour) | (rotl32(p2, 5) & kTwo);
-  p[4] = (p4b & kFour) | (rotl32(p2, 8) & kTwo);
-  p[5] = (rotl32(p4b, 4) & kFour) | (rotl32(p2, 9) & kTwo);
-  p[6] = (rotl32(p4b, 8) & kFour) | (rotl32(p2, 12) & kTwo);
-  p[7] = (rotl32(p4b, 12) & kFour) | (rotl32(p2, 13) & kTwo);
+// (a0, a1) += c, c a packed pair of fp32 constants held in a 64-bit register.
+__device__ __forceinline__ void fadd2c(float& a0, float& a1, uint64_t c) {
+  asm("{.reg .b64 a;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "add.rn.f32x2 a, a, %2;\n\t"
+      "mov.b64 {%0, %1}, a;}\n"
+      : "+f"(a0), "+f"(a1)
+      : "l"(c));
 }
 
-// int8 (offset binary): byte i of w is q + 128.  Output fp32 q for each byte:
-// the byte is placed in the low mantissa of 2^23 (exact 2^23 + q + 128), then
-// the constant is subtracted exactly.
-__device__ __forceinline__ void decode_int8_word(uint32_t w, float v[4]) {
-  constexpr float kBias = 8388608.0f + 128.0f;
-  v[0] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540)) - kBias;
-  v[1] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7541)) - kBias;
-  v[2] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7542)) - kBias;
-  v[3] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7543)) - kBias;
-}
-
-// acc += a * b with a, b the low (or high) bf16 of a pair register; fp32
-// accumulate, one rounding (mixed-precision FMA of sm_100).
-__device__ __forceinline__ void fma_bf16_lo(float& acc, uint32_t a, uint32_t b) {
-  asm("{.reg .b16 al, ah, bl, bh;\n\t"
-      "mov.b32 {al, ah}, %1;\n\t"
-      "mov.b32 {bl, bh}, %2;\n\t"
-      "fma.rn.f32.bf16 %0, al, bl, %0;}\n"
-      : "+f"(acc)
-      : "r"(a), "r"(b));
-}
-__device__ __forceinline__ void fma_bf16_hi(float& acc, uint32_t a, uint32_t b) {
-  asm("{.reg .b16 al, ah, bl, bh;\n\t"
-      "mov.b32 {al, ah}, %1;\n\t"
-      "mov.b32 {bl, bh}, %2;\n\t"
-      "fma.rn.f32.bf16 %0, ah, bh, %0;}\n"
-      : "+f"(acc)
-      : "r"(a), "r"(b));
-}
-// acc += a.lo * b.lo + a.hi * b.hi (two roundings, in that order).
-__device__ __forceinline__ void fma_bf16x2(float& acc, uint32_t a, uint32_t b) {
-  fma_bf16_lo(acc, a, b);
-  fma_bf16_hi(acc, a, b);
+// A packed pair of fp32 constants in a register whose value the compiler cannot
+// see, so that it stays live instead of being rebuilt from immediates at each use.
+__device__ __forceinline__ uint64_t opaque_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm volatile("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
 }
 
 // (acc0, acc1) += (w0 * x0, w1 * x1): packed fp32 FMA of sm_100 (one
@@ -92,9 +75,29 @@ __device__ __forceinline__ void ffma2(float& acc0, float& acc1, float w0, float 
       : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
 }
 
+// Packed fp32 pairs held as native 64-bit registers.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// acc += w * x on packed pairs (one fma.rn.f32x2).
+__device__ __forceinline__ void ffma2p(uint64_t& acc, uint64_t w, uint64_t x) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(w), "l"(x));
+}
+// packed pair + packed constant (one add.rn.f32x2)
+__device__ __forceinline__ uint64_t fadd2p(float lo, float hi, uint64_t c) {
+  uint64_t r;
+  asm("{.reg .b64 a;\n\tmov.b64 a, {%1, %2};\n\tadd.rn.f32x2 %0, a, %3;}" : "=l"(r) : "f"(lo), "f"(hi), "l"(c));
+  return r;
+}
+
 // Exact bf16 pair -> two floats.
 __device__ __forceinline__ float bf16_lo_f(uint32_t p) { return __uint_as_float(p << 16); }
-__device__ __forceinline__ float bf16_hi_f(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_hi_f(uint32_t p) { return __uint_as_float(lop_and(p, 0xFFFF0000u)); }
 
 // Pack two floats into a bf16 pair with round-to-nearest-even.
 __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
@@ -103,5 +106,101 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   return r;
 }
 
+// ------------------------------------------------------------------ int4
+// Word w holds q[8t + 2r + h] in bits 4r + 16h .. +3 (r = 0..3, h = 0..1).
+
+// bf16 bit pattern of 128.0 in both halves: OR-ing a 4-bit code into the low
+// mantissa bits gives the exact value 128 + q.
+constexpr uint32_t kBf16Magic128x2 = 0x43004300u;
+
+// Output p[r] = bf16 pair (128 + q[8t + 2r], 128 + q[8t + 2r + 1]), r = 0..3
+// (tensor-core operand form).
+__device__ __forceinline__ void decode_int4_word(uint32_t w, uint32_t p[4]) {
+  p[0] = lop_and_or(w, 0x000F000Fu, kBf16Magic128x2);
+  p[1] = lop_and_or(w >> 4, 0x000F000Fu, kBf16Magic128x2);
+  p[2] = lop_and_or(w >> 8, 0x000F000Fu, kBf16Magic128x2);
+  p[3] = lop_and_or(w >> 12, 0x000F000Fu, kBf16Magic128x2);
+}
+
+// fp32 exponent field of 2^e.
+__host__ __device__ constexpr uint32_t f32_exp_bits(int e) { return uint32_t(127 + e) << 23; }
+
+// CUDA-core form, two words at a time.  wa, wb are two int4 words.  For nibble
+// n of both words, one LOP3 per word masks the nibble and ORs the exponent of
+// 2^15 (the same register for every nibble), giving the two halves of an fp32
+// pair 2^15 + q * 2^(p - 8), p the nibble's mantissa bit; one packed subtract
+// of 2^15 leaves (q_a, q_b) * 2^(p - 8) exactly.  Nibbles at bits 0..19
+// (n = 0..4) are used in place; the three above (n = 5..7, bits 20..31) come
+// from the words shifted right by 12 (bits 8, 12, 16).  The activations are
+// pre-scaled by 2^(8 - p) to match (int4_x_scale_exp), so each product is
+// q * x exactly.
+constexpr uint32_t kInt4Magic = 0x47000000u;  // fp32 exponent field of 2^15
+__host__ __device__ constexpr int int4_nibble_bit(int n) { return n <= 4 ? 4 * n : 4 * n - 12; }
+// exponent of the activation pre-scale for nibble n
+__host__ __device__ constexpr int int4_x_scale_exp(int n) { return 8 - int4_nibble_bit(n); }
+
+struct Int4PairConsts {
+  uint32_t magic;  // kInt4Magic, kept in a register
+  uint64_t bias;   // packed (-2^15, -2^15)
+};
+__device__ __forceinline__ Int4PairConsts int4_pair_consts() {
+  Int4PairConsts c;
+  asm volatile("mov.b32 %0, %1;" : "=r"(c.magic) : "n"(kInt4Magic));
+  c.bias = opaque_f32x2(-0x1p15f, -0x1p15f);
+  return c;
+}
+
+// Packed pair (q_a, q_b) * 2^(p - 8) of nibble N (a template argument, so that
+// the mask is an immediate) of the words wa, wb (N <= 4) or of their
+// right-by-12 shifts (N >= 5, pass the shifted words).
+template <int N>
+__device__ __forceinline__ uint64_t int4_pair(uint32_t wa, uint32_t wb, const Int4PairConsts& c) {
+  constexpr uint32_t mask = 0xFu << int4_nibble_bit(N);
+  uint64_t r;
+  asm("{.reg .b32 lo, hi;\n\t"
+      ".reg .b64 p;\n\t"
+      "lop3.b32 lo, %1, %3, %4, 0xEA;\n\t"
+      "lop3.b32 hi, %2, %3, %4, 0xEA;\n\t"
+      "mov.b64 p, {lo, hi};\n\t"
+      "add.rn.f32x2 %0, p, %5;}"
+      : "=l"(r)
+      : "r"(wa), "r"(wb), "n"(mask), "r"(c.magic), "l"(c.bias));
+  return r;
+}
+
+// ------------------------------------------------------------------ FP6 e3m2
+// p2 is the 2-bit-plane word of 16 weights, p4a / p4b the two 4-bit-plane words
+// of its first and second 8 weights.  Output p[4c + j] = bf16 pair
+// (k = 8c + 2j, 8c + 2j + 1) holding code value * 2^-124 (subnormal for e = 0):
+// sign at bit 15, e2 e1 e0 at bits 9..7, m1 m0 at bits 6..5 of each half.
+__device__ __forceinline__ void decode_fp6_words(uint32_t p2, uint32_t p4a, uint32_t p4b, uint32_t p[8]) {
+  constexpr uint32_t kFour = 0x01E001E0u;  // bits 5..8 of each half: (e1 e0 m1 m0)
+  constexpr uint32_t kTwo = 0x82008200u;   // bits 15 and 9 of each half: sign, e2
+  p[0] = lop_and_or(p4a, kFour, lop_and(p2, kTwo));
+  p[1] = lop_and_or(rotl32(p4a, 4), kFour, lop_and(rotl32(p2, 1), kTwo));
+  p[2] = lop_and_or(rotl32(p4a, 8), kFour, lop_and(rotl32(p2, 4), kTwo));
+  p[3] = lop_and_or(rotl32(p4a, 12), kFour, lop_and(rotl32(p2, 5), kTwo));
+  p[4] = lop_and_or(p4b, kFour, lop_and(rotl32(p2, 8), kTwo));
+  p[5] = lop_and_or(rotl32(p4b, 4), kFour, lop_and(rotl32(p2, 9), kTwo));
+  p[6] = lop_and_or(rotl32(p4b, 8), kFour, lop_and(rotl32(p2, 12), kTwo));
+  p[7] = lop_and_or(rotl32(p4b, 12), kFour, lop_and(rotl32(p2, 13), kTwo));
+}
+
+// ------------------------------------------------------------------ int8
+// Offset binary: byte i of w is q + 128.  Output fp32 q for each byte: the byte
+// is placed in the low mantissa of 2^23 (exact 2^23 + q + 128, one PRMT), then
+// the constant is subtracted exactly (one packed subtract per pair, the pair
+// from int8_f32_bias()).
+__device__ __forceinline__ uint64_t int8_f32_bias() {
+  return opaque_f32x2(-(8388608.0f + 128.0f), -(8388608.0f + 128.0f));
+}
+__device__ __forceinline__ void decode_int8_word(uint32_t w, float v[4], uint64_t bias) {
+  v[0] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540));
+  v[1] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7541));
+  v[2] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7542));
+  v[3] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7543));
+  fadd2c(v[0], v[1], bias);
+  fadd2c(v[2], v[3], bias);
+}
 
 }  // namespace wq

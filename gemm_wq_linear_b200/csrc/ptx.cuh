@@ -69,6 +69,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Orders this thread's (and, after a barrier, its block's) generic-proxy shared
+// memory accesses before subsequent async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16-bit read-only global load, zero-extended into a 32-bit register by the
+// load itself (no instruction depends on the value until it is used).
+__device__ __forceinline__ uint32_t ld_nc_u16_u32(const uint16_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 // Bulk asynchronous copy global -> shared, completing `bytes` on the mbarrier.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

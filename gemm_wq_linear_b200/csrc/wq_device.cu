@@ -87,12 +87,23 @@ __global__ void unpack_debug_kernel(const uint8_t* __restrict__ packed, int fmt,
   if (fmt == WQ_INT4) {
     const uint4 w = *reinterpret_cast<const uint4*>(packed + size_t(n) * (K / 2) + k0 / 2);
     const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-    for (int q = 0; q < 4; ++q) {
-      uint32_t p[4];
-      decode_int4_word(words[q], p);
-      for (int r = 0; r < 4; ++r) {
-        v[8 * q + 2 * r] = bf16_lo_f(p[r]) - 128.f;
-        v[8 * q + 2 * r + 1] = bf16_hi_f(p[r]) - 128.f;
+    // the CUDA-core decoder (pairs of scaled q values from two words, rescaled
+    // here); the tensor-core decoder's bf16 pairs (128 + q) are checked by the
+    // GEMM parity tests
+    const Int4PairConsts c = int4_pair_consts();
+    for (int wp = 0; wp < 2; ++wp) {
+      const uint32_t wa = words[2 * wp], wb = words[2 * wp + 1];
+      const uint32_t sa = wa >> 12, sb = wb >> 12;
+      const uint64_t pr[8] = {int4_pair<0>(wa, wb, c), int4_pair<1>(wa, wb, c), int4_pair<2>(wa, wb, c),
+                              int4_pair<3>(wa, wb, c), int4_pair<4>(wa, wb, c), int4_pair<5>(sa, sb, c),
+                              int4_pair<6>(sa, sb, c), int4_pair<7>(sa, sb, c)};
+      for (int n = 0; n < 8; ++n) {
+        float lo, hi;
+        unpack2(pr[n], lo, hi);
+        const float unscale = ldexpf(1.0f, int4_x_scale_exp(n));
+        const int ka = 16 * wp + 2 * (n & 3) + (n >> 2);
+        v[ka] = lo * unscale;
+        v[ka + 8] = hi * unscale;
       }
     }
   } else if (fmt == WQ_FP6_E3M2) {
@@ -102,27 +113,22 @@ __global__ void unpack_debug_kernel(const uint8_t* __restrict__ packed, int fmt,
     const uint2 w2 = *reinterpret_cast<const uint2*>(p2 + size_t(n) * (K / 4) + k0 / 4);
     const uint32_t a4[4] = {w4.x, w4.y, w4.z, w4.w};
     const uint32_t a2[2] = {w2.x, w2.y};
-    const uint32_t one = 0x3F803F80u;  // bf16 (1, 1)
     for (int u = 0; u < 2; ++u) {
       uint32_t p[8];
       decode_fp6_words(a2[u], a4[2 * u], a4[2 * u + 1], p);
-      for (int c = 0; c < 2; ++c)
-        for (int j = 0; j < 4; ++j) {
-          // the compute path multiplies the scaled code with bf16 activations
-          // in fp32 and rescales by 2^124 at the end; mirror that with x = 1
-          float lo = 0.f, hi = 0.f;
-          fma_bf16_lo(lo, p[4 * c + j], one);
-          fma_bf16_hi(hi, p[4 * c + j], one);
-          v[16 * u + 8 * c + 2 * j] = lo * 0x1p124f;
-          v[16 * u + 8 * c + 2 * j + 1] = hi * 0x1p124f;
-        }
+      // the compute path widens the scaled code pairs to fp32 exactly and
+      // rescales by 2^124 at the end; mirror that
+      for (int i = 0; i < 8; ++i) {
+        v[16 * u + 2 * i] = bf16_lo_f(p[i]) * 0x1p124f;
+        v[16 * u + 2 * i + 1] = bf16_hi_f(p[i]) * 0x1p124f;
+      }
     }
   } else if (fmt == WQ_INT8) {
     const uint8_t* base = packed + size_t(n) * K + k0;
     for (int q = 0; q < 4; ++q) {
       const uint2 w = *reinterpret_cast<const uint2*>(base + 8 * q);
-      decode_int8_word(w.x, v + 8 * q);
-      decode_int8_word(w.y, v + 8 * q + 4);
+      decode_int8_word(w.x, v + 8 * q, int8_f32_bias());
+      decode_int8_word(w.y, v + 8 * q + 4, int8_f32_bias());
     }
   } else {
     const uint16_t* base = reinterpret_cast<const uint16_t*>(packed) + size_t(n) * K + k0;

@@ -1,5 +1,5 @@
 // Swap-AB weight-only-quantized GEMM on the sm_100a tensor cores (tcgen05),
-// for the decode linear at 5 <= M <= 32.
+// for the decode linear at 5 <= M <= 32 (and on request at M <= 4).
 //
 //   D[n, m] = sum_k deq(W)[n, k] * x[m, k]     (the weight tile is the MMA's M = 128,
 //                                               the activation rows its N = MPAD)
@@ -11,16 +11,20 @@
 // laid out for B200:
 //
 //  * warp 0 streams packed weight tiles (128 rows x 128 k) and the matching
-//    activation tile with 2-D tensor copies into an mbarrier ring;
-//  * warps 2-5 (one thread per weight row) decode their row in registers and
-//    write exact bf16 code values into an A tile in the canonical K-major
-//    128-byte-swizzle layout (int4 as 128 + q, FP6 as its e3m2 value, int8 as q);
-//  * one thread of warp 1 issues tcgen05.mma (kind::f16, 128 x MPAD x 16) with
-//    A and B from shared memory and the fp32 accumulator in tensor memory;
-//  * the same four warps read the accumulator with tcgen05.ld and apply the
-//    scales in fp32: per output channel at the end (int8, FP6), or per group as
-//    each group's partial product completes (int4: y += s_g D_g + (z_g - 128 s_g) X_g,
-//    X_g the sum of x over the group);
+//    activation tile with 2-D tensor copies into an mbarrier ring (~200 KB);
+//  * sixteen dequant warps (four per TMEM lane quadrant, one k-quarter each)
+//    decode their quarter-row in registers into exact bf16 code values (int4
+//    as 128 + q, FP6 as its e3m2 value, int8 as q) and store them straight into
+//    a tensor-memory A tile with tcgen05.st;
+//  * three issuing warps take every third k-block each and issue tcgen05.mma
+//    (kind::f16, 128 x MPAD x 16, A from tensor memory, B = activations from
+//    shared memory) into fp32 accumulators in tensor memory, one commit per
+//    block (a lone issuing thread is limited to one MMA per ~50 cycles and a
+//    commit costs it several hundred, so one issuer cannot keep up);
+//  * scales are applied in fp32: per output channel at the end (int8, FP6), or
+//    per group as each group's partial product completes (int4:
+//    y += s_g D_g + (z_g - 128 s_g) X_g, X_g the sum of x over the group),
+//    a few blocks behind the MMAs so that no warp waits for the tensor core;
 //  * K is split over the CTAs of a thread-block cluster; the partial results are
 //    summed in rank order through distributed shared memory (no global scratch).
 //
@@ -42,8 +46,10 @@ namespace gemm {
 
 constexpr int kBM = 128;   // weight rows per tile (MMA M)
 constexpr int kBK = 128;   // k per pipeline stage
-constexpr int kDqWarps = 16;                 // dequant / epilogue warps: 4 per TMEM lane quadrant
-constexpr int kThreads = 32 * (2 + kDqWarps);  // + producer warp + MMA warp
+constexpr int kIssuers = 3;   // MMA-issuing warps; each owns every third k-block
+constexpr int kDqWarps = 16;  // dequant / epilogue warps: 4 per TMEM lane quadrant
+constexpr int kDq0 = 1 + kIssuers;                    // first dequant warp
+constexpr int kThreads = 32 * (kDq0 + kDqWarps);      // + producer warp
 constexpr int kACols = kBK / 2;  // TMEM columns of one A tile (two bf16 per column)
 constexpr int kXsSlots = 8;      // int4: ring of per-block group sums of x
 
@@ -123,6 +129,7 @@ __device__ __forceinline__ void dequant_quarter(const uint8_t* W, int r, int u, 
       }
     }
   } else if constexpr (FMT == WQ_INT8) {
+    const uint64_t bias = int8_f32_bias();
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const uint4 w = *reinterpret_cast<const uint4*>(W + swz<128>(r, 2 * u + c));
@@ -130,7 +137,7 @@ __device__ __forceinline__ void dequant_quarter(const uint8_t* W, int r, int u, 
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         float f[4];
-        decode_int8_word(ws[t], f);
+        decode_int8_word(ws[t], f, bias);
         p[8 * c + 2 * t] = pack_bf16x2_rn(f[0], f[1]);
         p[8 * c + 2 * t + 1] = pack_bf16x2_rn(f[2], f[3]);
       }
@@ -160,8 +167,18 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
   return v;
 }
 
-// MPAD: MMA N (activation rows padded to a multiple of 8); MV <= MPAD: rows the
+// MPAD: MMA N (activation rows padded to a multiple of 16); MV <= MPAD: rows the
 // epilogue carries (the valid rows rounded up to a power of two).
+//
+// Warp roles: 0 streams tiles; 1 .. kIssuers issue the MMAs of the k-blocks
+// j == warp - 1 (mod kIssuers) (one thread each: a single issuing thread spends
+// about 50 cycles per tcgen05.mma and several hundred per commit, so the issue
+// is spread over warps); the kDqWarps others dequantize (warp quadrant q owns
+// TMEM lanes 32 q .., k-quarter u of every block) and run the epilogue.
+//
+// One commit per block, on mdone[stage]: it frees the stage's tiles for the
+// producer, the block's A tile for the dequant warps and (int4) tells the
+// folding warps that the block's group accumulators are complete.
 template <int FMT, int MPAD, int MV>
 __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_constant__ GemmParams a) {
   using L = Layout<FMT, MPAD>;
@@ -169,20 +186,22 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   constexpr int NA = L::kNumA;
   constexpr bool kInt4 = FMT == WQ_INT4;
   constexpr bool kTmemA = FMT != WQ_BF16;  // bf16 weights are the A operand in shared memory as loaded
+  // bf16 needs no dequantization and far fewer MMAs per byte: one issuer (the
+  // shared-memory-operand form is only issued from a single thread)
+  constexpr int kIss = kTmemA ? kIssuers : 1;
+  static_assert(NW > NA, "the ring must be deeper than the A tiles");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment of the tiles (swizzle atoms and descriptors need it)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + L::kRingBytes);
   uint64_t* full_w = bars;             // [NW]  tensor copies landed
-  uint64_t* empty_w = full_w + NW;     // [NW]  MMA finished with the stage
-  uint64_t* afull = empty_w + NW;      // [NA]  A tile written to TMEM
-  uint64_t* aempty = afull + NA;       // [NA]  MMA finished with the A tile
-  uint64_t* dfull = aempty + NA;       // [4]   accumulator (block-)buffer complete
-  uint64_t* dempty = dfull + 4;        // [4]   int4: accumulator block-buffer drained
+  uint64_t* mdone = full_w + NW;       // [NW]  MMAs of the stage's block completed
+  uint64_t* afull = mdone + NW;        // [NA]  A tile written to TMEM
+  uint64_t* dempty = afull + NA;       // [4]   int4: accumulator block-buffer folded
   uint64_t* xready = dempty + 4;       // [kXsSlots] int4: group sums of x of a block written
-  uint64_t* done = xready + kXsSlots;  // [1]   every MMA of the CTA completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* done = xready + kXsSlots;  // [kIssuers] every MMA of an issuer completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + kIssuers);
   int* issued_slot = reinterpret_cast<int*>(tmem_slot + 1);
   float* xs = reinterpret_cast<float*>(tmem_slot + 4);  // int4: [kXsSlots][4 groups][MV] group sums of x
   // writer warps of the group sums: entries (activation row, 8-k chunk) = MV x 16
@@ -199,27 +218,23 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   const int nkb = max(0, min(a.kb_per_split, KB - kb0));
   const int g = kInt4 ? a.groupsize : kBK;
   const int gpb = kBK / g;  // groups per k-block (int4)
-  // TMEM columns: [0, NA * 64) A tiles, then accumulators
+  // TMEM columns: [0, NA * 64) A tiles, then accumulators (int4: ndb block-buffers
+  // of gpb groups; otherwise one per issuer)
   constexpr uint32_t kDCol = NA * kACols;
-  const int ndb = kInt4 ? (gpb * MPAD <= 64 ? 4 : 2) : 1;  // int4 accumulator block-buffers
+  const int ndb = kInt4 ? min(4, 256 / (gpb * MPAD)) : 1;
+  const int lag = ndb - 1;  // int4: block j is folded while block j + lag is dequantized
   const uint32_t tmem_cols = a.tmem_cols;
 
   if (a.pdl) pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int i = 0; i < NW; ++i) {
       mbar_init(&full_w[i], 1);
-      mbar_init(&empty_w[i], 1);
+      mbar_init(&mdone[i], 1);
     }
-    for (int i = 0; i < NA; ++i) {
-      mbar_init(&afull[i], kDqWarps);
-      mbar_init(&aempty[i], 1);
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&dfull[i], 1);
-      mbar_init(&dempty[i], 4);
-    }
+    for (int i = 0; i < NA; ++i) mbar_init(&afull[i], kDqWarps);
+    for (int i = 0; i < 4; ++i) mbar_init(&dempty[i], 4);
     for (int i = 0; i < kXsSlots; ++i) mbar_init(&xready[i], kXsWarps);
-    mbar_init(done, 1);
+    for (int i = 0; i < kIssuers; ++i) mbar_init(&done[i], 1);
     *issued_slot = 0;
     fence_mbar_init();
   }
@@ -248,10 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
         tma_load_2d_nohint(st + Fmt<FMT>::kWBytes, &a.tm_x, kx, 0, &full_w[j % NW]);
         tma_load_2d_nohint(st + Fmt<FMT>::kWBytes + MPAD * 128, &a.tm_x, kx + 64, 0, &full_w[j % NW]);
       };
-      int j = 0;
+      int j = 0, s = 0;
+      uint32_t ph = 0;
       for (; j < nkb; ++j) {
-        const int s = j % NW;
-        if (!mbar_wait(&empty_w[s], ((j / NW) & 1) ^ 1)) {
+        // the stage's previous block (j - NW) must be finished by the tensor core
+        if (!mbar_wait(&mdone[s], ph ^ 1u)) {
           failed = true;
           break;
         }
@@ -274,19 +290,29 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
           pdl_wait();  // x may come from the previous kernel
           for (int j2 = 0; j2 < T0; ++j2) issue_x(j2);
         }
+        if (++s == NW) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       *issued_slot = j;
       if (failed && a.pdl && j < T0) pdl_wait();
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp <= kIssuers) {
+    // ------------------------------------------------------------ MMA issuers
+    const int iss = warp - 1;
+    if (lane == 0 && iss < kIss) {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, MPAD);
-      for (int j = 0; j < nkb && !failed; ++j) {
+      for (int j = iss; j < nkb; j += kIss) {
         const int s = j % NW;
         const int ai = j % NA;
         if (!mbar_wait(kTmemA ? &afull[ai] : &full_w[s], kTmemA ? ((j / NA) & 1) : ((j / NW) & 1))) {
+          failed = true;
+          break;
+        }
+        const int db = j & (ndb - 1);
+        if (kInt4 && !mbar_wait(&dempty[db], ((j / ndb) & 1) ^ 1)) {
           failed = true;
           break;
         }
@@ -304,61 +330,56 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
         };
         if constexpr (kInt4) {
           // every group of the block into its own MPAD-column accumulator
-          const int db = j & (ndb - 1);
-          if (!mbar_wait(&dempty[db], ((j / ndb) & 1) ^ 1)) {
-            failed = true;
-            break;
-          }
-          tc_fence_after();
           const int kvalid = min(kBK, a.K - (kb0 + j) * kBK);
           for (int gi = 0; gi < gpb && gi * g < kvalid; ++gi)
             for (int kk = gi * (g / 16); kk < (gi + 1) * (g / 16); ++kk)
               mma_step(tmem + kDCol + (db * gpb + gi) * MPAD, kk, kk != gi * (g / 16));
-          mma_commit(&dfull[db]);
         } else {
 #pragma unroll 1
-          for (int kk = 0; kk < kBK / 16; ++kk) mma_step(tmem + kDCol, kk, (j | kk) != 0);
+          for (int kk = 0; kk < kBK / 16; ++kk) mma_step(tmem + kDCol + iss * MPAD, kk, (j != iss) || kk != 0);
         }
-        if constexpr (kTmemA) mma_commit(&aempty[ai]);  // A tile free
-        mma_commit(&empty_w[s]);
+        mma_commit(&mdone[s]);
       }
-      if (!kInt4) mma_commit(&dfull[0]);  // accumulator complete
-      mma_commit(done);
+      mma_commit(&done[iss]);  // every MMA of this issuer complete
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ dequant + epilogue
-    // warp 2 + d: TMEM lane quadrant q = warp % 4 (rows 32 q ..), k-quarter u = d / 4
-    const int d = warp - 2;
+    // warp kDq0 + d: TMEM lane quadrant q = warp % 4 (rows 32 q ..), k-quarter u = d / 4
+    const int d = warp - kDq0;
     const int u = d >> 2;
     const int r = 32 * (warp & 3) + lane;
     const int n = n0 + r;
-    const int dtid = threadIdx.x - 64;  // 0 .. 511 (warp d holds entries 32 d ..)
+    const int dtid = threadIdx.x - 32 * kDq0;  // 0 .. 511 (warp d holds entries 32 d ..)
     const uint32_t trow = uint32_t(32 * (warp & 3)) << 16;  // TMEM lane base of this warp
     const int G = kInt4 ? a.K / g : 0;
     if (a.pdl) pdl_wait();
-    // int4: scale and zero of this row for the groups of the block this warp folds
-    float sz_s[4], sz_z[4];
+    // int4: raw 16-bit scale and zero of this row for the groups of the block this
+    // warp group folds next (it has at most one block pending).  Nothing uses the
+    // loaded registers until the fold, several blocks later, so the loads' latency
+    // never stalls the dequantization.
+    uint32_t sz_s[4], sz_z[4];
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi) sz_s[gi] = sz_z[gi] = 0u;
     auto load_sz = [&](int j) {
       if constexpr (kInt4) {
         const int gbase = (kb0 + j) * (kBK / g);
 #pragma unroll
         for (int gi = 0; gi < 4; ++gi) {
-          const bool ok = gi < gpb && n < a.N && (kb0 + j) * kBK + gi * g < a.K;
-          const size_t gidx = size_t(n) * G + gbase + gi;
-          sz_s[gi] = ok ? bf16f(a.scales[gidx]) : 0.f;
-          sz_z[gi] = ok ? bf16f(a.zeros[gidx]) : 0.f;
+          if (gi < gpb && n < a.N && (kb0 + j) * kBK + gi * g < a.K) {
+            const size_t gidx = size_t(n) * G + gbase + gi;
+            sz_s[gi] = ld_nc_u16_u32(a.scales + gidx);
+            sz_z[gi] = ld_nc_u16_u32(a.zeros + gidx);
+          }
         }
       }
     };
     // int4: fold the group accumulators of block j into acc (warps with u == j % 4)
-    auto fold_block = [&](int j) {
+    auto fold_block = [&](int j) -> bool {
       if constexpr (kInt4) {
         const int db = j & (ndb - 1);
-        if (!mbar_wait(&dfull[db], (j / ndb) & 1) || !mbar_wait(&xready[j % kXsSlots], (j / kXsSlots) & 1)) {
-          failed = true;
-          return;
-        }
+        if (!mbar_wait(&mdone[j % NW], (j / NW) & 1) || !mbar_wait(&xready[j % kXsSlots], (j / kXsSlots) & 1))
+          return false;
         tc_fence_after();
         const int kvalid = min(kBK, a.K - (kb0 + j) * kBK);
 #pragma unroll
@@ -368,17 +389,20 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
             uint32_t dv[LD];
             tmem_ld_32x32b<LD>(tmem + trow + kDCol + (db * gpb + gi) * MPAD, dv);
             tmem_ld_wait();
-            const float sc = sz_s[gi];
-            const float zc = fmaf(-128.f, sc, sz_z[gi]);
+            const float sc = __uint_as_float(sz_s[gi] << 16);
+            const float zc = __uint_as_float(sz_z[gi] << 16);
             const float* xg = xs + ((j % kXsSlots) * 4 + gi) * MV;
+            // accumulators hold sum((128 + q) x): s * D + (z - 128 s) * X
+            const float zc2 = fmaf(-128.f, sc, zc);
 #pragma unroll
-            for (int m = 0; m < MV; ++m) acc[m] = fmaf(sc, __uint_as_float(dv[m]), fmaf(zc, xg[m], acc[m]));
+            for (int m = 0; m < MV; ++m) acc[m] = fmaf(sc, __uint_as_float(dv[m]), fmaf(zc2, xg[m], acc[m]));
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&dempty[db]);
       }
+      return true;
     };
     if constexpr (kTmemA) {
       for (int j = 0; j < nkb && !failed; ++j) {
@@ -389,7 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
         const uint8_t* st = ring + size_t(s) * L::kStage;
         uint32_t pv[16];
         dequant_quarter<FMT>(st, r, u, pv);
-        if (!mbar_wait(&aempty[ai], ((j / NA) & 1) ^ 1)) { failed = true; break; }
+        // the A tile's previous block (j - NA) must be finished by the tensor core
+        if (j >= NA && !mbar_wait(&mdone[(j - NA) % NW], ((j - NA) / NW) & 1)) { failed = true; break; }
         tc_fence_after();
         tmem_st_32x32b_x16(tmem + trow + ai * kACols + 16 * u, pv);
         tmem_st_wait();
@@ -398,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
         if (lane == 0) mbar_arrive(&afull[ai]);
         if constexpr (kInt4) {
           // group sums of x for this block from the B tile (the first kXsWarps
-          // warps; entry e = 16 m + c, chunk c of 8 k), then fold block j - 1
+          // warps; entry e = 16 m + c, chunk c of 8 k)
           if (d < kXsWarps) {
             const uint8_t* xt = st + Fmt<FMT>::kWBytes;
             const int e = dtid;
@@ -416,27 +441,26 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(&xready[j % kXsSlots]);
           }
-          if (j >= 1 && ((j - 1) & 3) == u) fold_block(j - 1);
+          const int jf = j - lag;
+          if (jf >= 0 && (jf & 3) == u && !fold_block(jf)) { failed = true; break; }
         }
       }
       if constexpr (kInt4) {
-        if (!failed && nkb >= 1 && ((nkb - 1) & 3) == u) fold_block(nkb - 1);
+        for (int jf = max(0, nkb - lag); jf < nkb && !failed; ++jf)
+          if ((jf & 3) == u && !fold_block(jf)) failed = true;
       }
     }
     if constexpr (!kInt4) {
-      if (!failed && u == 0) {
-        if (mbar_wait(&dfull[0], 0)) {
+      // issuer u's accumulator (issuers without a block hold nothing)
+      if (!failed && u < kIss && u < nkb) {
+        if (mbar_wait(&done[u], 0)) {
           tc_fence_after();
           constexpr int LD = MV <= 8 ? 8 : MV;
           uint32_t dv[LD];
-          tmem_ld_32x32b<LD>(tmem + trow + kDCol, dv);
+          tmem_ld_32x32b<LD>(tmem + trow + kDCol + u * MPAD, dv);
           tmem_ld_wait();
-          float sc = 1.f;
-          if (n < a.N) {
-            if constexpr (FMT == WQ_INT8 || FMT == WQ_FP6_E3M2) sc = fp16f(a.scales[n]);
-          }
 #pragma unroll
-          for (int m = 0; m < MV; ++m) acc[m] = __uint_as_float(dv[m]) * sc;
+          for (int m = 0; m < MV; ++m) acc[m] = __uint_as_float(dv[m]);
         } else {
           failed = true;
         }
@@ -452,31 +476,34 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
       // let every issued copy land and every issued MMA finish before leaving
       const int issued = *issued_slot;
       for (int j = max(0, issued - NW); j < issued; ++j) mbar_wait(&full_w[j % NW], (j / NW) & 1);
-      mbar_wait(done, 0);
+      for (int i = 0; i < kIss; ++i) mbar_wait(&done[i], 0);
     }
   }
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, tmem_cols);
 
-  const bool epi = warp >= 2;
-  const int u = (warp - 2) >> 2;
+  const bool epi = warp >= kDq0;
+  const int u = (warp - kDq0) >> 2;
   const int r = 32 * (warp & 3) + lane;
   const int n = n0 + r;
-  // int4: the four k-quarter warp groups each folded a quarter of the blocks;
-  // partials meet in the (now idle) ring
+  // the four k-quarter warp groups each hold a partial (int4: a quarter of the
+  // blocks folded; otherwise issuer u's accumulator); they meet in the idle ring
   float* red = reinterpret_cast<float*>(ring);  // [3][128][MV]
-  if (kInt4) {
-    if (epi && u > 0) {
+  if (epi && u > 0) {
 #pragma unroll
-      for (int m = 0; m < MV; ++m) red[((u - 1) * 128 + r) * MV + m] = acc[m];
-    }
-    __syncthreads();
-    if (epi && u == 0) {
+    for (int m = 0; m < MV; ++m) red[((u - 1) * 128 + r) * MV + m] = acc[m];
+  }
+  __syncthreads();
+  if (epi && u == 0) {
 #pragma unroll
-      for (int q = 0; q < 3; ++q)
+    for (int q = 0; q < 3; ++q)
 #pragma unroll
-        for (int m = 0; m < MV; ++m) acc[m] += red[(q * 128 + r) * MV + m];
+      for (int m = 0; m < MV; ++m) acc[m] += red[(q * 128 + r) * MV + m];
+    if constexpr (FMT == WQ_INT8 || FMT == WQ_FP6_E3M2) {
+      const float sc = n < a.N ? fp16f(a.scales[n]) : 0.f;
+#pragma unroll
+      for (int m = 0; m < MV; ++m) acc[m] *= sc;
     }
   }
   const bool out = epi && u == 0;
@@ -490,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   }
   // split-K over the cluster: partials through distributed shared memory
   constexpr int MV4 = MV < 4 ? 4 : MV;                          // row pitch of the partial buffer (16-byte units)
-  float* part = reinterpret_cast<float*>(ring) + 3 * 128 * MV;  // [128][MV4], after the int4 partials
+  float* part = reinterpret_cast<float*>(ring) + 3 * 128 * MV;  // [128][MV4], after the quarter partials
   if (out) {
 #pragma unroll
     for (int m = 0; m < MV4; m += 4)
@@ -528,18 +555,27 @@ static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int 
   GemmParams p = p0;
   const int tiles = (p.N + gemm::kBM - 1) / gemm::kBM;
   const int KB = (p.K + gemm::kBK - 1) / gemm::kBK;
-  // split K over a cluster so that about one CTA per SM is busy; int4 keeps each
-  // CTA's k range at most 4096 (the per-group x sums live in shared memory)
-  int S = (sm_count + tiles / 2) / tiles;
-  if (S > 8) S = 8;
-  if (S > KB) S = KB;
-  if (S < 1) S = 1;
-  int kbps = (KB + S - 1) / S;
-  S = (KB + kbps - 1) / kbps;
+  // split K over a cluster of S CTAs (one CTA per SM): pick S so that the
+  // rounds of CTAs times the k-blocks per CTA (plus a fixed cost of about two
+  // blocks for filling and draining the pipeline) is smallest
+  int S = 1, kbps = KB;
+  long best = -1;
+  for (int s = 1; s <= 8 && s <= KB; ++s) {
+    const int bps = (KB + s - 1) / s;
+    const int s_eff = (KB + bps - 1) / bps;
+    const long rounds = (long(tiles) * s_eff + sm_count - 1) / sm_count;
+    const long cost = rounds * (bps + 2);
+    if (best < 0 || cost < best) {
+      best = cost;
+      S = s_eff;
+      kbps = bps;
+    }
+  }
   p.splits = S;
   p.kb_per_split = kbps;
   p.tmem_cols = 512;  // A tiles (4 x 64 columns) + accumulators (<= 256 columns)
-  const size_t small = 1024 + 64 * 8 + 64 + size_t(gemm::kXsSlots * 4 * MV) * 4;
+  const size_t small = 1024 + size_t(2 * L::kNumW + L::kNumA + 4 + gemm::kXsSlots + gemm::kIssuers) * 8 + 64 +
+                       size_t(gemm::kXsSlots * 4 * MV) * 4;
   const size_t smem = L::kRingBytes + small;
   static_assert(L::kRingBytes >= (3 * 128 * MV + 128 * (MV < 4 ? 4 : MV)) * 4,
                 "reduction buffers must fit the idle ring");

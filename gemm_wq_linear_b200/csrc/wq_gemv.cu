@@ -22,9 +22,11 @@
 //    memory, scaled and rounded to bf16.
 //
 // Dequantization arithmetic (fp32 accumulation):
-//  * int4: decoded value 128 + q (bf16); per lane and group
-//    s * sum(x (128 + q)) + (z - 128 s) * sum(x)  =  sum(x (q s + z)).
-//  * FP6: decoded value v * 2^-124 (bf16, subnormal for e = 0); y = 2^124 s_n sum.
+//  * int4: decoded value q * 2^(p - 8) against activations scaled by 2^(8 - p)
+//    (p the nibble's bit position, decode.cuh): exact products q x; per lane
+//    and group s * sum(x q) + z * sum(x)  =  sum(x (q s + z)).
+//  * FP6: decoded value v * 2^-124 (bf16 pair widened to fp32, subnormal for
+//    e = 0); y = 2^124 s_n sum.
 //  * int8: fp32 q; y = s_n sum.   bf16: plain products.
 #include "wq_internal.h"
 #include "wq_kernels.cuh"
@@ -51,8 +53,8 @@ struct GemvFmt<WQ_FP6_E3M2> {
 };
 template <>
 struct GemvFmt<WQ_INT8> {
-  static constexpr int kLaneK = 8;
-  static constexpr int kRowBytes = 256;
+  static constexpr int kLaneK = 16;
+  static constexpr int kRowBytes = 512;
 };
 template <>
 struct GemvFmt<WQ_BF16> {
@@ -62,9 +64,14 @@ struct GemvFmt<WQ_BF16> {
 
 constexpr int kRB = 32;                 // rows per stage (one per producer lane)
 constexpr int kConsumerWarps = 8;
-constexpr int kGemvThreads = 32 * (1 + kConsumerWarps);
-// Two CTAs per SM while the activations of one chunk fit the register budget, one beyond.
-__host__ __device__ constexpr int gemv_ctas_per_sm(int mm) { return mm <= 2 ? 2 : 1; }
+// M <= 2: a producer warp keeps the ring full ahead of the eight consumer warps
+// (two CTAs per SM at M = 1, one at M = 2).  M >= 3 (the activations of a chunk
+// need more registers): one CTA per SM of eight consumer warps and no producer,
+// so each thread may hold up to 255 registers; the last warp to finish a stage
+// refills its slot.
+__host__ __device__ constexpr bool gemv_has_producer(int mm) { return mm <= 2; }
+__host__ __device__ constexpr int gemv_ctas_per_sm(int mm) { return mm <= 1 ? 2 : 1; }
+__host__ __device__ constexpr int gemv_threads(int mm) { return 32 * (kConsumerWarps + (gemv_has_producer(mm) ? 1 : 0)); }
 
 template <int FMT, int MM>
 struct GemvLayout {
@@ -73,13 +80,7 @@ struct GemvLayout {
   static constexpr int kStageBytes = (kRB * GemvFmt<FMT>::kRowBytes + MM * kXBytes + 127) / 128 * 128;
 };
 
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 __device__ __forceinline__ float fp16_bits_to_float(uint16_t b) { return __half2float(__ushort_as_half(b)); }
-__device__ __forceinline__ uint16_t ld_u16(const uint16_t* p) {
-  uint16_t v;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-  return v;
-}
 
 // Packed bytes of `kc` weights of one row for the format.
 template <int FMT>
@@ -90,64 +91,106 @@ __host__ __device__ __forceinline__ uint32_t row_chunk_bytes(int kc) {
   return uint32_t(kc) * 2;
 }
 
-// Per-lane activation registers of one chunk, for MM rows of x, as fp32 (exact).
+// Per-lane activation registers of one chunk, for MM rows of x, as packed fp32
+// pairs matching the weight pairs the decoder produces:
+//  * int4: pair 8 w + n = (k_a, k_a + 8) with k_a = 16 w + 2 (n & 3) + (n >> 2)
+//    (nibble n of words 2w and 2w + 1), scaled by 2^(8 - p(n)) (decode.cuh);
+//  * other formats: pair i = (2 i, 2 i + 1).
+// All conversions and scalings are exact (powers of two).
 template <int FMT, int MM>
 struct XRegs {
-  float v[MM][GemvFmt<FMT>::kLaneK];
-  float xsum[MM];  // int4: sum of the lane's 32 activations
+  uint64_t v2[MM][GemvFmt<FMT>::kLaneK / 2];
+  float xsum[MM];  // int4: sum of the lane's 32 activations (unscaled)
 };
 
+__host__ __device__ constexpr float pow2f(int e) {
+  return e >= 0 ? float(1u << e) : 1.0f / float(1u << -e);
+}
+
+// Lanes past the end of K (last chunk) get zeros: their weights are the tensor
+// copy's zero fill, so every product is zero without a per-lane branch.
 template <int FMT, int MM>
-__device__ __forceinline__ void load_x_smem(XRegs<FMT, MM>& xr, const uint8_t* xs, int lane) {
+__device__ __forceinline__ void load_x_smem(XRegs<FMT, MM>& xr, const uint8_t* xs, int lane, bool valid) {
   using L = GemvLayout<FMT, MM>;
+  constexpr int LK = GemvFmt<FMT>::kLaneK;
 #pragma unroll
   for (int m = 0; m < MM; ++m) {
-    const uint8_t* base = xs + m * L::kXBytes + lane * GemvFmt<FMT>::kLaneK * 2;
+    const uint8_t* base = xs + m * L::kXBytes + lane * LK * 2;
+    float xf[LK];
 #pragma unroll
-    for (int q = 0; q < GemvFmt<FMT>::kLaneK / 8; ++q) {
-      const uint4 v = *reinterpret_cast<const uint4*>(base + 16 * q);
+    for (int q = 0; q < LK / 8; ++q) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) v = *reinterpret_cast<const uint4*>(base + 16 * q);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        xr.v[m][8 * q + 2 * i] = bf16_lo_f(w[i]);
-        xr.v[m][8 * q + 2 * i + 1] = bf16_hi_f(w[i]);
+        xf[8 * q + 2 * i] = bf16_lo_f(w[i]);
+        xf[8 * q + 2 * i + 1] = bf16_hi_f(w[i]);
       }
     }
     if constexpr (FMT == WQ_INT4) {
+#pragma unroll
+      for (int wp = 0; wp < 2; ++wp)
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+          const int ka = 16 * wp + 2 * (n & 3) + (n >> 2);
+          constexpr float kScale[8] = {pow2f(int4_x_scale_exp(0)), pow2f(int4_x_scale_exp(1)),
+                                       pow2f(int4_x_scale_exp(2)), pow2f(int4_x_scale_exp(3)),
+                                       pow2f(int4_x_scale_exp(4)), pow2f(int4_x_scale_exp(5)),
+                                       pow2f(int4_x_scale_exp(6)), pow2f(int4_x_scale_exp(7))};
+          xr.v2[m][8 * wp + n] = pack2(xf[ka] * kScale[n], xf[ka + 8] * kScale[n]);
+        }
       float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < GemvFmt<FMT>::kLaneK; i += 2) {
-        s0 += xr.v[m][i];
-        s1 += xr.v[m][i + 1];
+      for (int i = 0; i < LK; i += 2) {
+        s0 += xf[i];
+        s1 += xf[i + 1];
       }
       xr.xsum[m] = s0 + s1;
+    } else {
+#pragma unroll
+      for (int i = 0; i < LK / 2; ++i) xr.v2[m][i] = pack2(xf[2 * i], xf[2 * i + 1]);
     }
   }
 }
 
+template <int FMT>
+struct DecodeConsts {
+  Int4PairConsts i4;
+  uint64_t i8;
+};
+template <int FMT>
+__device__ __forceinline__ DecodeConsts<FMT> make_decode_consts() {
+  DecodeConsts<FMT> d;
+  if constexpr (FMT == WQ_INT4) d.i4 = int4_pair_consts();
+  if constexpr (FMT == WQ_INT8) d.i8 = int8_f32_bias();
+  return d;
+}
+
 // Lane partial of one row-chunk for every activation row.  `w` points at the
-// lane's row in shared memory (FP6: `w2p` at its 2-bit plane).  Decoded bf16
-// pairs are widened to fp32 exactly (a shift and a mask) and accumulated with the
-// packed fp32 FMA; the two halves of each pair use separate accumulators.
+// lane's row in shared memory (FP6: `w2p` at its 2-bit plane).  Decoded values
+// are exact fp32 pairs and accumulate with the packed fp32 FMA (one pair of
+// accumulators per activation row).
 template <int FMT, int MM>
 __device__ __forceinline__ void lane_dot(const uint8_t* w, const uint8_t* w2p, int lane, const XRegs<FMT, MM>& xr,
-                                         float acc[MM]) {
-  float a0[MM], a1[MM];
+                                         const DecodeConsts<FMT>& dc, float acc[MM]) {
+  uint64_t ac[MM];
 #pragma unroll
-  for (int m = 0; m < MM; ++m) a0[m] = a1[m] = 0.f;
+  for (int m = 0; m < MM; ++m) ac[m] = 0ull;
   if constexpr (FMT == WQ_INT4) {
     const uint4 wv = *reinterpret_cast<const uint4*>(w + lane * 16);
     const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t p[4];
-      decode_int4_word(words[q], p);
+    for (int wp = 0; wp < 2; ++wp) {
+      const uint32_t wa = words[2 * wp], wb = words[2 * wp + 1];
+      const uint32_t sa = wa >> 12, sb = wb >> 12;
+      const uint64_t v[8] = {int4_pair<0>(wa, wb, dc.i4), int4_pair<1>(wa, wb, dc.i4), int4_pair<2>(wa, wb, dc.i4),
+                             int4_pair<3>(wa, wb, dc.i4), int4_pair<4>(wa, wb, dc.i4), int4_pair<5>(sa, sb, dc.i4),
+                             int4_pair<6>(sa, sb, dc.i4), int4_pair<7>(sa, sb, dc.i4)};
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float lo = bf16_lo_f(p[r]), hi = bf16_hi_f(p[r]);
+      for (int n = 0; n < 8; ++n)
 #pragma unroll
-        for (int m = 0; m < MM; ++m) ffma2(a0[m], a1[m], lo, hi, xr.v[m][8 * q + 2 * r], xr.v[m][8 * q + 2 * r + 1]);
-      }
+        for (int m = 0; m < MM; ++m) ffma2p(ac[m], v[n], xr.v2[m][8 * wp + n]);
     }
   } else if constexpr (FMT == WQ_FP6_E3M2) {
     const uint4 w4 = *reinterpret_cast<const uint4*>(w + lane * 16);
@@ -160,206 +203,236 @@ __device__ __forceinline__ void lane_dot(const uint8_t* w, const uint8_t* w2p, i
       decode_fp6_words(a2[v], a4[2 * v], a4[2 * v + 1], p);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float lo = bf16_lo_f(p[j]), hi = bf16_hi_f(p[j]);
+        const uint64_t pw = pack2(bf16_lo_f(p[j]), bf16_hi_f(p[j]));
 #pragma unroll
-        for (int m = 0; m < MM; ++m) ffma2(a0[m], a1[m], lo, hi, xr.v[m][16 * v + 2 * j], xr.v[m][16 * v + 2 * j + 1]);
+        for (int m = 0; m < MM; ++m) ffma2p(ac[m], pw, xr.v2[m][8 * v + j]);
       }
     }
   } else if constexpr (FMT == WQ_INT8) {
-    const uint2 wv = *reinterpret_cast<const uint2*>(w + lane * 8);
-    float v[8];
-    decode_int8_word(wv.x, v);
-    decode_int8_word(wv.y, v + 4);
+    const uint4 wv = *reinterpret_cast<const uint4*>(w + lane * 16);
+    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-    for (int i = 0; i < 8; i += 2)
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t wq = words[q];
+      const uint64_t p0 = fadd2p(__uint_as_float(__byte_perm(wq, 0x4B000000u, 0x7540)),
+                                 __uint_as_float(__byte_perm(wq, 0x4B000000u, 0x7541)), dc.i8);
+      const uint64_t p1 = fadd2p(__uint_as_float(__byte_perm(wq, 0x4B000000u, 0x7542)),
+                                 __uint_as_float(__byte_perm(wq, 0x4B000000u, 0x7543)), dc.i8);
 #pragma unroll
-      for (int m = 0; m < MM; ++m) ffma2(a0[m], a1[m], v[i], v[i + 1], xr.v[m][i], xr.v[m][i + 1]);
+      for (int m = 0; m < MM; ++m) {
+        ffma2p(ac[m], p0, xr.v2[m][2 * q]);
+        ffma2p(ac[m], p1, xr.v2[m][2 * q + 1]);
+      }
+    }
   } else {
     const uint4 wv = *reinterpret_cast<const uint4*>(w + lane * 16);
     const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float lo = bf16_lo_f(ww[i]), hi = bf16_hi_f(ww[i]);
+      const uint64_t pw = pack2(bf16_lo_f(ww[i]), bf16_hi_f(ww[i]));
 #pragma unroll
-      for (int m = 0; m < MM; ++m) ffma2(a0[m], a1[m], lo, hi, xr.v[m][2 * i], xr.v[m][2 * i + 1]);
+      for (int m = 0; m < MM; ++m) ffma2p(ac[m], pw, xr.v2[m][i]);
     }
   }
 #pragma unroll
-  for (int m = 0; m < MM; ++m) acc[m] = a0[m] + a1[m];
+  for (int m = 0; m < MM; ++m) {
+    float lo, hi;
+    unpack2(ac[m], lo, hi);
+    acc[m] = lo + hi;
+  }
 }
 
+// Position of a stage in the CTA's sequence: ring slot and phase parity, row
+// block and (rotated) chunk.  Stages run chunk-major over the row blocks.
+struct StagePos {
+  int slot;
+  uint32_t phase;
+  int rb;
+  int c;
+};
+__device__ __forceinline__ void advance(StagePos& p, int NS, int NRB, int C) {
+  if (++p.rb == NRB) {
+    p.rb = 0;
+    p.c = (p.c + 1 == C) ? 0 : p.c + 1;
+  }
+  if (++p.slot == NS) {
+    p.slot = 0;
+    p.phase ^= 1u;
+  }
+}
 
 template <int FMT, int MM>
-__global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kernel(const __grid_constant__ GemvParams a) {
+__global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_kernel(const __grid_constant__ GemvParams a) {
   using F = GemvFmt<FMT>;
   using L = GemvLayout<FMT, MM>;
   constexpr int kChunkK = L::kChunkK;
+  constexpr bool kProducer = gemv_has_producer(MM);
   extern __shared__ __align__(1024) uint8_t smem[];
 
   const int NS = a.stages;
   uint8_t* ring = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(NS) * L::kStageBytes);
-  uint64_t* empty = full + NS;
-  int* drain_info = reinterpret_cast<int*>(empty + NS);  // [0] stages issued
-  float* part = reinterpret_cast<float*>(drain_info + 4);  // [C][R][MM]
+  uint64_t* empty = full + NS;                          // [NS] warps finished reading the slot's stage
+  int* done_cnt = reinterpret_cast<int*>(empty + NS);  // [NS] arrivals counted, to elect the refilling warp
+  int* last_issued = done_cnt + NS;                    // [NS] stage last issued into the slot
+  float* part = reinterpret_cast<float*>(last_issued + NS + (NS & 1));  // [C][R][MM], 8-byte aligned
   const int C = (a.K + kChunkK - 1) / kChunkK;
   const int n0 = blockIdx.x * a.rows_per_cta;
   const int R = min(a.rows_per_cta, a.N - n0);
   const int NRB = (R + kRB - 1) / kRB;
   const int T = C * NRB;
-  // stages run chunk-major over the CTA's row blocks; each CTA starts at a
-  // different chunk so that concurrent CTAs fetch different parts of x
+  // each CTA starts at a different chunk so that concurrent CTAs fetch
+  // different parts of x
   const int c_rot = blockIdx.x % C;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint64_t policy = l2_policy_evict_first();
+
+  // Issue the tensor copies of one stage into its slot (one thread).  The x of a
+  // chunk travels with the chunk's first stage only.
+  auto issue_w = [&](const StagePos& p) {
+    const int rows = min(kRB, R - p.rb * kRB);
+    const int nbox = (rows + a.box_rows - 1) / a.box_rows;
+    const int kc = min(kChunkK, a.K - p.c * kChunkK);
+    mbar_arrive_expect_tx(&full[p.slot],
+                          uint32_t(nbox * a.box_rows * F::kRowBytes) + (p.rb == 0 ? MM * uint32_t(kc) * 2 : 0u));
+    uint8_t* st = ring + size_t(p.slot) * L::kStageBytes;
+    const int row0 = n0 + p.rb * kRB;
+    for (int b = 0; b < nbox; ++b) {
+      const int row = row0 + b * a.box_rows;
+      if constexpr (FMT == WQ_FP6_E3M2) {
+        tma_load_2d(st + b * a.box_rows * 512, &a.tm_w, p.c * (512 / 4), row, &full[p.slot], policy);
+        tma_load_2d(st + kRB * 512 + b * a.box_rows * 256, &a.tm_w2, p.c * (256 / 4), row, &full[p.slot], policy);
+      } else {
+        tma_load_2d(st + b * a.box_rows * F::kRowBytes, &a.tm_w, p.c * (F::kRowBytes / 4), row, &full[p.slot], policy);
+      }
+    }
+  };
+  auto issue_x = [&](const StagePos& p) {
+    if (p.rb != 0) return;
+    const int kc = min(kChunkK, a.K - p.c * kChunkK);
+    for (int m = 0; m < MM; ++m)
+      bulk_g2s(ring + size_t(p.slot) * L::kStageBytes + kRB * F::kRowBytes + m * L::kXBytes,
+               a.x + size_t(m) * a.K + size_t(p.c) * kChunkK, uint32_t(kc) * 2, &full[p.slot]);
+  };
 
   if (a.pdl) pdl_launch_dependents();
+  const int T0 = min(T, NS);
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
+      done_cnt[s] = 0;
+      last_issued[s] = -1;
     }
-    drain_info[0] = 0;
     fence_mbar_init();
+    prefetch_tmap(&a.tm_w);
+    if (FMT == WQ_FP6_E3M2) prefetch_tmap(&a.tm_w2);
+    if constexpr (!kProducer) {
+      // first ring fill: weights at once; x after the previous kernel (which may
+      // write it) has finished, under programmatic dependent launch
+      StagePos q = {0, 0u, 0, c_rot};
+      for (int t = 0; t < T0; ++t) {
+        issue_w(q);
+        last_issued[q.slot] = t;
+        advance(q, NS, NRB, C);
+      }
+      if (a.pdl) pdl_wait();
+      q = {0, 0u, 0, c_rot};
+      for (int t = 0; t < T0; ++t) {
+        issue_x(q);
+        advance(q, NS, NRB, C);
+      }
+    }
   }
   __syncthreads();
 
   bool failed = false;
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    const uint64_t policy = l2_policy_evict_first();
-    const int T0 = min(T, NS);
-    const int BH = a.box_rows;
+  if (kProducer && warp == 0) {
+    // ------------------------------------------------------------ producer (M = 1)
     if (lane == 0) {
-      prefetch_tmap(&a.tm_w);
-      if (FMT == WQ_FP6_E3M2) prefetch_tmap(&a.tm_w2);
-    }
-    auto issue_x = [&](int t) {
-      const int s = t % NS;
-      if (t % NRB != 0) return;  // x of a chunk travels with the chunk's first stage only
-      int c = t / NRB + c_rot;
-      c = c >= C ? c - C : c;
-      const int kc = min(kChunkK, a.K - c * kChunkK);
-      if (lane < MM)
-        bulk_g2s(ring + size_t(s) * L::kStageBytes + kRB * F::kRowBytes + lane * L::kXBytes,
-                 a.x + size_t(lane) * a.K + size_t(c) * kChunkK, uint32_t(kc) * 2, &full[s]);
-    };
-    int t = 0;
-    for (; t < T; ++t) {
-      const int s = t % NS;
-      if (!mbar_wait(&empty[s], ((t / NS) & 1) ^ 1)) {
-        failed = true;
-        break;
-      }
-      const int ci = t / NRB;
-      const int rb = t - ci * NRB;
-      const int c = ci + c_rot >= C ? ci + c_rot - C : ci + c_rot;
-      const int rows = min(kRB, R - rb * kRB);
-      const int nbox = (rows + BH - 1) / BH;
-      const int kc = min(kChunkK, a.K - c * kChunkK);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], uint32_t(nbox * BH * F::kRowBytes) + (rb == 0 ? MM * uint32_t(kc) * 2 : 0u));
-        uint8_t* st = ring + size_t(s) * L::kStageBytes;
-        for (int b = 0; b < nbox; ++b) {
-          const int row = n0 + rb * kRB + b * BH;
-          if constexpr (FMT == WQ_FP6_E3M2) {
-            tma_load_2d(st + b * BH * 512, &a.tm_w, c * (512 / 4), row, &full[s], policy);
-            tma_load_2d(st + kRB * 512 + b * BH * 256, &a.tm_w2, c * (256 / 4), row, &full[s], policy);
-          } else {
-            tma_load_2d(st + b * BH * F::kRowBytes, &a.tm_w, c * (F::kRowBytes / 4), row, &full[s], policy);
+      StagePos p = {0, 0u, 0, c_rot};
+      for (int t = 0; t < T; ++t) {
+        if (!mbar_wait(&empty[p.slot], p.phase ^ 1u)) {
+          failed = true;
+          break;
+        }
+        issue_w(p);
+        last_issued[p.slot] = t;
+        if (t >= T0 || !a.pdl) issue_x(p);
+        if (t == T0 - 1 && a.pdl) {
+          // weights of the first ring fill are in flight; x may be written by
+          // the previous kernel, so wait for it before fetching x
+          pdl_wait();
+          StagePos q = {0, 0u, 0, c_rot};
+          for (int t2 = 0; t2 < T0; ++t2) {
+            issue_x(q);
+            advance(q, NS, NRB, C);
           }
         }
+        advance(p, NS, NRB, C);
       }
-      __syncwarp();
-      if (t >= T0 || !a.pdl) issue_x(t);
-      if (t == T0 - 1 && a.pdl) {
-        // weights of the first ring fill are in flight; x may be written by
-        // the previous kernel, so wait for it before fetching x
-        pdl_wait();
-        for (int t2 = 0; t2 < T0; ++t2) issue_x(t2);
-      }
+      if (failed && a.pdl) pdl_wait();
     }
-    if (lane == 0) drain_info[0] = t;
-    if (failed && a.pdl && t < T0) pdl_wait();
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ consumers
-    const int cw = warp - 1;
-    const int ctid = threadIdx.x - 32;
+    const int cw = kProducer ? warp - 1 : warp;
     if (a.pdl) pdl_wait();
     int cur_c = -1;
     XRegs<FMT, MM> xr;
+    const DecodeConsts<FMT> dc = make_decode_consts<FMT>();
     constexpr int J = kRB / kConsumerWarps;  // rows of a stage this warp takes (4)
-    // int4 scales / zeros of this warp's rows, fetched kPf stages ahead (a small
-    // register ring), so their global latency hides behind the ring
-    constexpr int kPf = (FMT == WQ_INT4) ? 3 : 1;
-    uint32_t szq[kPf][J];
-    auto fetch_sz = [&](int t, uint32_t* dst) {
+    const int gshift = (FMT == WQ_INT4) ? __ffs(a.groupsize) - 1 : 0;
+    const int G = (FMT == WQ_INT4) ? (a.K >> gshift) : 0;
+    // int4: raw 16-bit scale and zero of this warp's rows at the lane's group,
+    // fetched one stage ahead into the other of two register sets; the load
+    // zero-extends, so no instruction touches them before the fold a stage later
+    auto fetch_sz = [&](const StagePos& p, uint32_t (&ds)[J], uint32_t (&dz)[J]) {
       if constexpr (FMT == WQ_INT4) {
-        if (t >= T) return;
-        const int ci = t / NRB;
-        const int rb = t - ci * NRB;
-        const int c = ci + c_rot >= C ? ci + c_rot - C : ci + c_rot;
-        const int rows = min(kRB, R - rb * kRB);
-        const int k0 = c * kChunkK + lane * F::kLaneK;
+        const int rows = min(kRB, R - p.rb * kRB);
+        const int k0 = p.c * kChunkK + lane * F::kLaneK;
         if (k0 >= a.K) return;
-        const int G = a.K / a.groupsize;
+        const size_t off = size_t(n0 + p.rb * kRB + cw) * G + (k0 >> gshift);
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-          const int i = cw + j * kConsumerWarps;
-          if (i < rows) {
-            const size_t gi = size_t(n0 + rb * kRB + i) * G + k0 / a.groupsize;
-            dst[j] = uint32_t(ld_u16(a.scales + gi)) | (uint32_t(ld_u16(a.zeros + gi)) << 16);
+          if (cw + j * kConsumerWarps < rows) {
+            ds[j] = ld_nc_u16_u32(a.scales + off + size_t(j * kConsumerWarps) * G);
+            dz[j] = ld_nc_u16_u32(a.zeros + off + size_t(j * kConsumerWarps) * G);
           }
         }
       }
     };
-    if constexpr (FMT == WQ_INT4) {
-#pragma unroll
-      for (int d = 0; d < kPf; ++d) fetch_sz(d, szq[d]);
-    }
-    for (int t = 0; t < T; ++t) {
-      const int s = t % NS;
-      uint32_t sz_cur[J];
-      if constexpr (FMT == WQ_INT4) {
-        // rotate the register ring: slot 0 is this stage
-#pragma unroll
-        for (int j = 0; j < J; ++j) sz_cur[j] = szq[0][j];
-#pragma unroll
-        for (int d = 0; d + 1 < kPf; ++d)
-#pragma unroll
-          for (int j = 0; j < J; ++j) szq[d][j] = szq[d + 1][j];
-        fetch_sz(t + kPf, szq[kPf - 1]);
+    // one stage: prefetch the next stage's scales, wait for this stage's tiles,
+    // dot products of the warp's rows, hand the slot back (the last warp out
+    // refills it with stage t + NS), reduce across lanes
+    auto stage = [&](int t, StagePos& p, StagePos& pr, bool has_next, const uint32_t (&ss)[J],
+                     const uint32_t (&zz)[J], uint32_t (&ss_next)[J], uint32_t (&zz_next)[J]) -> bool {
+      StagePos nx = p;
+      advance(nx, NS, NRB, C);
+      if (has_next) fetch_sz(nx, ss_next, zz_next);
+      if (!mbar_wait(&full[p.slot], p.phase)) return false;
+      const int rows = min(kRB, R - p.rb * kRB);
+      const uint8_t* st = ring + size_t(p.slot) * L::kStageBytes;
+      if (p.c != cur_c) {
+        load_x_smem<FMT, MM>(xr, st + kRB * F::kRowBytes, lane, p.c * kChunkK + lane * F::kLaneK < a.K);
+        cur_c = p.c;
       }
-      if (!mbar_wait(&full[s], (t / NS) & 1)) {
-        failed = true;
-        break;
-      }
-      const int ci = t / NRB;
-      const int rb = t - ci * NRB;
-      const int c = ci + c_rot >= C ? ci + c_rot - C : ci + c_rot;
-      const int rows = min(kRB, R - rb * kRB);
-      const int k0 = c * kChunkK + lane * F::kLaneK;
-      const bool active = k0 < a.K;
-      const uint8_t* st = ring + size_t(s) * L::kStageBytes;
-      if (c != cur_c) {
-        if (active) {
-          load_x_smem<FMT, MM>(xr, st + kRB * F::kRowBytes, lane);
-        }
-        cur_c = c;
-      }
-      // all J rows of this warp at once: independent chains interleave
+      // all J rows of this warp at once: independent chains interleave (the row
+      // test is uniform across the warp)
       float acc[J][MM];
 #pragma unroll
       for (int j = 0; j < J; ++j) {
         const int i = cw + j * kConsumerWarps;
-        if (active && i < rows) {
+        if (i < rows) {
           if constexpr (FMT == WQ_FP6_E3M2)
-            lane_dot<FMT, MM>(st + i * 512, st + kRB * 512 + i * 256, lane, xr, acc[j]);
+            lane_dot<FMT, MM>(st + i * 512, st + kRB * 512 + i * 256, lane, xr, dc, acc[j]);
           else
-            lane_dot<FMT, MM>(st + i * F::kRowBytes, nullptr, lane, xr, acc[j]);
+            lane_dot<FMT, MM>(st + i * F::kRowBytes, nullptr, lane, xr, dc, acc[j]);
           if constexpr (FMT == WQ_INT4) {
-            const float sc = bf16_bits_to_float(uint16_t(sz_cur[j] & 0xFFFFu));
-            const float zc = fmaf(-128.f, sc, bf16_bits_to_float(uint16_t(sz_cur[j] >> 16)));
+            // sum over the lane's 32 k (one group): s * sum(q x) + z * sum(x)
+            const float sc = __uint_as_float(ss[j] << 16);
+            const float zc = __uint_as_float(zz[j] << 16);
 #pragma unroll
             for (int m = 0; m < MM; ++m) acc[j][m] = fmaf(sc, acc[j][m], zc * xr.xsum[m]);
           }
@@ -368,8 +441,28 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
           for (int m = 0; m < MM; ++m) acc[j][m] = 0.f;
         }
       }
+      // every lane's shared-memory reads of the stage are done: release them on
+      // the slot's empty barrier
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);  // shared memory of the stage no longer read
+      bool ok = true;
+      if (lane == 0) {
+        mbar_arrive(&empty[p.slot]);
+        if constexpr (!kProducer) {
+          // the counter elects the last warp, which waits for the barrier
+          // (acquiring every warp's reads) and refills the slot with stage t + NS
+          if (atomicAdd(&done_cnt[p.slot], 1) == kConsumerWarps - 1) {
+            done_cnt[p.slot] = 0;
+            ok = mbar_wait(&empty[p.slot], p.phase);
+            if (ok && t + NS < T) {
+              fence_proxy_async_shared();
+              issue_w(pr);
+              issue_x(pr);
+              last_issued[pr.slot] = t + NS;
+            }
+          }
+        }
+      }
+      if (!kProducer && !__shfl_sync(0xFFFFFFFFu, int(ok), 0)) return false;
       // transposed butterfly: 6 shuffles reduce the 4 rows; lane 8j holds row j
       static_assert(J == 4, "reduction below assumes 4 rows per warp and stage");
 #pragma unroll
@@ -388,20 +481,41 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(MM)) gemv_kerne
         if ((lane & 7) == 0) {
           const int j = lane >> 3;  // 2 * (bit 4) + (bit 3)
           const int i = cw + j * kConsumerWarps;
-          if (i < rows) part[(size_t(c) * R + rb * kRB + i) * MM + m] = kv;
+          if (i < rows) part[(size_t(p.c) * R + p.rb * kRB + i) * MM + m] = kv;
         }
+      }
+      p = nx;
+      advance(pr, NS, NRB, C);
+      return true;
+    };
+    uint32_t sA[J], zA[J], sB[J], zB[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) sA[j] = zA[j] = sB[j] = zB[j] = 0u;
+    StagePos p = {0, 0u, 0, c_rot};
+    StagePos pr = p;  // position of stage t + NS
+    for (int i = 0; i < NS; ++i) advance(pr, NS, NRB, C);
+    fetch_sz(p, sA, zA);
+    for (int t = 0; t < T; t += 2) {
+      if (!stage(t, p, pr, t + 1 < T, sA, zA, sB, zB)) {
+        failed = true;
+        break;
+      }
+      if (t + 1 < T && !stage(t + 1, p, pr, t + 2 < T, sB, zB, sA, zA)) {
+        failed = true;
+        break;
       }
     }
   }
 
   // ---------------------------------------------------------------- epilogue
-  __syncthreads();
   const bool any_failed = __syncthreads_or(failed);
   if (any_failed) {
     // wait (bounded) until every copy issued into the ring has landed, then leave
     if (threadIdx.x == 0) {
-      const int issued = drain_info[0];
-      for (int t = max(0, issued - NS); t < issued; ++t) mbar_wait(&full[t % NS], (t / NS) & 1);
+      for (int s = 0; s < NS; ++s) {
+        const int u = last_issued[s];
+        if (u >= 0) mbar_wait(&full[s], (u / NS) & 1);
+      }
     }
     return;
   }
@@ -441,13 +555,13 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   if (R < kBoxRows) R = kBoxRows;
   p.rows_per_cta = R;
   p.box_rows = kBoxRows;
-  const size_t fixed = 16 * 8 + 16 + size_t(C) * R * MM * 4;
+  const size_t fixed = 8 * 24 + 16 + size_t(C) * R * MM * 4;
   if (fixed + 2 * size_t(L::kStageBytes) > 200 * 1024) return cudaErrorInvalidValue;
   int stages = fixed < kGemvSmemBudget ? int((kGemvSmemBudget - fixed) / L::kStageBytes) : 2;
   if (stages > 8) stages = 8;
   if (stages < 2) stages = 2;
   p.stages = stages;
-  const size_t smem = size_t(stages) * L::kStageBytes + size_t(stages) * 16 + 16 + size_t(C) * R * MM * 4;
+  const size_t smem = size_t(stages) * L::kStageBytes + size_t(stages) * 24 + 16 + size_t(C) * R * MM * 4;
 
   // tensor maps: rows of packed bytes viewed as 32-bit elements, one chunk per box
   cudaError_t e;
@@ -467,7 +581,7 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   const int grid = (p.N + R - 1) / R;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kGemvThreads);
+  cfg.blockDim = dim3(gemv_threads(MM));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
