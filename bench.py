@@ -22,7 +22,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -84,57 +83,95 @@ def layer_seed(idx):
 
 
 # ------------------------------------------------------------------ clocks
-CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+# clock event reason bits (NVML): the ones that reject a measurement, and the
+# power cap (kept and noted)
+_REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Polls the GPU's SM clock, max clock, clock event reasons and power through
+    NVML every 2 ms while the timed region runs (a background thread that only
+    reads)."""
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"wq_clocks_{os.getpid()}.csv")
+    def __init__(self, torch_index):
+        self.samples = []
+        self.handle = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it instead of clocks
+            self.err = f"nvml unavailable: {type(e).__name__}"
+        self.stop = None
+
+    def _run(self):
+        nv, h = self.nv, self.handle
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((sm, rs, pw))
+            except Exception:
+                pass
+            self.stop.wait(0.002)
 
     def __enter__(self):
-        try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        if self.handle is not None:
+            import threading
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            time.sleep(0.15)
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.f.close()
+        if self.stop is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for ln in f:
-                p = [s.strip() for s in ln.split(",")]
-                if len(p) >= 9 and p[1].replace(".", "").isdigit():
-                    rows.append(p)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows]
-        mx = max(float(r[2]) for r in rows)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        reasons = sorted({name for (_, rs, _) in self.samples for bit, name in _REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_max": max(s[2] for s in self.samples)}
+
+
+# ------------------------------------------------------------------ measured DRAM traffic
+KERNEL_SOURCES = ("gemm_wq_linear_b200/csrc/wq_gemv.cu", "gemm_wq_linear_b200/csrc/decode.cuh",
+                  "gemm_wq_linear_b200/csrc/ptx.cuh")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload):
+    """DRAM bytes (read + write) per launch of the GEMV kernel for `workload`, from
+    the committed ncu summary, or None when there is none or the kernel sources
+    changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"gemv_{workload}_traffic.md")
+    try:
+        with open(path) as f:
+            kv = dict(ln.split(":", 1) for ln in f if ln.startswith(("traffic_bytes_per_launch:", "kernel_source_hash:")))
+    except OSError:
+        return None
+    if kv.get("kernel_source_hash", "").strip() != kernel_source_hash():
+        return None
+    return float(kv["traffic_bytes_per_launch"])
 
 
 # ------------------------------------------------------------------ peaks
@@ -230,7 +267,7 @@ def oracle_sample_run(layers, budget_s):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="wq", choices=["wq", "reference"])
     ap.add_argument("--workload", default="llama2-7b-int4-m1")
@@ -238,12 +275,17 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline")
     ap.add_argument("--layers-detail", action="store_true", help="also time each layer alone")
+    ap.add_argument("--layer", default=None, help="run only the layer with this label (for profiling one kernel)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
     world, rank, local = dist_setup(args)
     layers = workload_layers(args.workload)
+    if args.layer:
+        layers = [ly for ly in layers if ly[0] == args.layer]
+        if not layers:
+            raise SystemExit(f"no layer {args.layer} in {args.workload}")
     total_bytes = sum(algo_bytes(f, g, K, N, M) for (_, f, g, K, N, M) in layers)
     metric = "effective weight GB/s (algorithmic bytes / device time), M=1..32 decode linear"
 
@@ -395,7 +437,9 @@ def main():
                    "parallelism": f"replicas x{world}"},
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None},
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": None if args.layer else measured_traffic(args.workload),
+                     "algorithmic_bytes_per_launch": total_bytes / len(bufs)},
         "layer_us_alone": layer_us,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},

@@ -52,6 +52,7 @@ constexpr int kDq0 = 1 + kIssuers;                    // first dequant warp
 constexpr int kThreads = 32 * (kDq0 + kDqWarps);      // + producer warp
 constexpr int kACols = kBK / 2;  // TMEM columns of one A tile (two bf16 per column)
 constexpr int kXsSlots = 8;      // int4: ring of per-block group sums of x
+constexpr int kSzSlots = 8;      // int4: ring of staged scale / zero boxes
 
 template <int FMT>
 struct Fmt;
@@ -79,7 +80,10 @@ struct Layout {
   // dequantized A tiles live in tensor memory (4 x 64 columns); shared memory
   // holds only the packed-weight / activation ring, ~200 KB of it in flight
   static constexpr int kNumA = 4;
-  static constexpr int kNumW0 = (200 * 1024) / kStage;
+  // int4: ring of kSzSlots scale / zero boxes (8 groups x 128 rows of each)
+  static constexpr int kSzSlotBytes = FMT == WQ_INT4 ? 2 * 128 * 8 * 2 : 0;
+  static constexpr int kSzBytes = kSzSlots * kSzSlotBytes;
+  static constexpr int kNumW0 = (200 * 1024 - kSzBytes) / kStage;
   static constexpr int kNumW = kNumW0 > 16 ? 16 : kNumW0;
   static constexpr int kRingBytes = kNumW * kStage;
   static_assert(kStage % 1024 == 0, "stages must keep 1024-byte alignment");
@@ -194,14 +198,17 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   // 1024-byte alignment of the tiles (swizzle atoms and descriptors need it)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + L::kRingBytes);
+  uint8_t* szring = ring + L::kRingBytes;  // int4: [kSzSlots][s: 128 x 8][z: 128 x 8] bf16
+  uint64_t* bars = reinterpret_cast<uint64_t*>(szring + L::kSzBytes);
   uint64_t* full_w = bars;             // [NW]  tensor copies landed
   uint64_t* mdone = full_w + NW;       // [NW]  MMAs of the stage's block completed
   uint64_t* afull = mdone + NW;        // [NA]  A tile written to TMEM
   uint64_t* dempty = afull + NA;       // [4]   int4: accumulator block-buffer folded
   uint64_t* xready = dempty + 4;       // [kXsSlots] int4: group sums of x of a block written
   uint64_t* done = xready + kXsSlots;  // [kIssuers] every MMA of an issuer completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + kIssuers);
+  uint64_t* szfull = done + kIssuers;  // [kSzSlots] int4: scale / zero box landed
+  uint64_t* szfree = szfull + kSzSlots;  // [kSzSlots] int4: every block of the box folded
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(szfree + kSzSlots);
   int* issued_slot = reinterpret_cast<int*>(tmem_slot + 1);
   float* xs = reinterpret_cast<float*>(tmem_slot + 4);  // int4: [kXsSlots][4 groups][MV] group sums of x
   // writer warps of the group sums: entries (activation row, 8-k chunk) = MV x 16
@@ -235,6 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
     for (int i = 0; i < 4; ++i) mbar_init(&dempty[i], 4);
     for (int i = 0; i < kXsSlots; ++i) mbar_init(&xready[i], kXsWarps);
     for (int i = 0; i < kIssuers; ++i) mbar_init(&done[i], 1);
+    for (int i = 0; i < kSzSlots; ++i) {
+      mbar_init(&szfull[i], 1);
+      mbar_init(&szfree[i], 4 * (8 / gpb));  // the fold of each of the box's blocks, 4 warps each
+    }
     *issued_slot = 0;
     fence_mbar_init();
   }
@@ -284,6 +295,22 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
         } else {
           tma_load_2d(st, &a.tm_w, kb * kBK, n0, &full_w[s], policy);
           tma_load_2d(st + kBM * 128, &a.tm_w, kb * kBK + 64, n0, &full_w[s], policy);
+        }
+        if constexpr (kInt4) {
+          // the scale / zero box of blocks j .. j + spb - 1 (8 groups of every row)
+          const int spb = 8 / gpb;
+          if (a.sz_tma && j % spb == 0) {
+            const int box = j / spb;
+            const int zs = box % kSzSlots;
+            if (!mbar_wait(&szfree[zs], ((box / kSzSlots) & 1) ^ 1)) {
+              failed = true;
+              break;
+            }
+            mbar_arrive_expect_tx(&szfull[zs], uint32_t(L::kSzSlotBytes));
+            uint8_t* dst = szring + zs * L::kSzSlotBytes;
+            tma_load_2d_nohint(dst, &a.tm_s, (kb0 + j) * gpb, n0, &szfull[zs]);
+            tma_load_2d_nohint(dst + L::kSzSlotBytes / 2, &a.tm_z, (kb0 + j) * gpb, n0, &szfull[zs]);
+          }
         }
         if (j >= T0 || !a.pdl) issue_x(j);
         if (j == T0 - 1 && a.pdl) {
@@ -380,27 +407,58 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
         const int db = j & (ndb - 1);
         if (!mbar_wait(&mdone[j % NW], (j / NW) & 1) || !mbar_wait(&xready[j % kXsSlots], (j / kXsSlots) & 1))
           return false;
+        const int spb = 8 / gpb;
+        const int box = j / spb;
+        const int zs = box % kSzSlots;
+        if (a.sz_tma) {
+          // this row's scales and zeros of the block, from the staged box
+          if (!mbar_wait(&szfull[zs], (box / kSzSlots) & 1)) return false;
+          const uint16_t* sp = reinterpret_cast<const uint16_t*>(szring + zs * L::kSzSlotBytes) + r * 8 + (j % spb) * gpb;
+          const uint16_t* zp = sp + L::kSzSlotBytes / 4;
+#pragma unroll
+          for (int gi = 0; gi < 4; ++gi) {
+            if (gi < gpb) {
+              sz_s[gi] = sp[gi];
+              sz_z[gi] = zp[gi];
+            }
+          }
+        }
         tc_fence_after();
         const int kvalid = min(kBK, a.K - (kb0 + j) * kBK);
+        // the group accumulators of the block are read in batches of GB groups
+        // with one wait per batch (each wait is a round trip to tensor memory)
+        constexpr int LD = MV <= 8 ? 8 : MV;  // columns loaded per group
+        constexpr int GB = 4 * LD <= 32 ? 4 : (2 * LD <= 32 ? 2 : 1);
 #pragma unroll
-        for (int gi = 0; gi < 4; ++gi) {
-          if (gi < gpb && gi * g < kvalid) {
-            constexpr int LD = MV <= 8 ? 8 : MV;  // columns loaded per group
-            uint32_t dv[LD];
-            tmem_ld_32x32b<LD>(tmem + trow + kDCol + (db * gpb + gi) * MPAD, dv);
+        for (int gi0 = 0; gi0 < 4; gi0 += GB) {
+          if (gi0 < gpb) {
+            uint32_t dv[GB][LD];
+#pragma unroll
+            for (int b = 0; b < GB; ++b)
+              if (gi0 + b < gpb && (gi0 + b) * g < kvalid)
+                tmem_ld_32x32b<LD>(tmem + trow + kDCol + (db * gpb + gi0 + b) * MPAD, dv[b]);
             tmem_ld_wait();
-            const float sc = __uint_as_float(sz_s[gi] << 16);
-            const float zc = __uint_as_float(sz_z[gi] << 16);
-            const float* xg = xs + ((j % kXsSlots) * 4 + gi) * MV;
-            // accumulators hold sum((128 + q) x): s * D + (z - 128 s) * X
-            const float zc2 = fmaf(-128.f, sc, zc);
 #pragma unroll
-            for (int m = 0; m < MV; ++m) acc[m] = fmaf(sc, __uint_as_float(dv[m]), fmaf(zc2, xg[m], acc[m]));
+            for (int b = 0; b < GB; ++b) {
+              const int gi = gi0 + b;
+              if (gi < gpb && gi * g < kvalid) {
+                const float sc = __uint_as_float(sz_s[gi] << 16);
+                const float zc = __uint_as_float(sz_z[gi] << 16);
+                const float* xg = xs + ((j % kXsSlots) * 4 + gi) * MV;
+                // accumulators hold sum((128 + q) x): s * D + (z - 128 s) * X
+                const float zc2 = fmaf(-128.f, sc, zc);
+#pragma unroll
+                for (int m = 0; m < MV; ++m) acc[m] = fmaf(sc, __uint_as_float(dv[b][m]), fmaf(zc2, xg[m], acc[m]));
+              }
+            }
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dempty[db]);
+        if (lane == 0) {
+          mbar_arrive(&dempty[db]);
+          if (a.sz_tma) mbar_arrive(&szfree[zs]);
+        }
       }
       return true;
     };
@@ -408,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
       for (int j = 0; j < nkb && !failed; ++j) {
         const int s = j % NW;
         const int ai = j % NA;
-        if (kInt4 && (j & 3) == u) load_sz(j);
+        if (kInt4 && !a.sz_tma && (j & 3) == u) load_sz(j);
         if (!mbar_wait(&full_w[s], (j / NW) & 1)) { failed = true; break; }
         const uint8_t* st = ring + size_t(s) * L::kStage;
         uint32_t pv[16];
@@ -555,16 +613,30 @@ static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int 
   GemmParams p = p0;
   const int tiles = (p.N + gemm::kBM - 1) / gemm::kBM;
   const int KB = (p.K + gemm::kBK - 1) / gemm::kBK;
+  // int4: scales and zeros are staged by tensor copies of 8-group boxes when the
+  // row pitch (K / g bf16) is a multiple of 16 bytes and both arrays are 16-byte
+  // aligned; a box spans spb k-blocks, so every split starts on a box boundary
+  int spb = 1;
+  p.sz_tma = 0;
+  if constexpr (FMT == WQ_INT4) {
+    const int G = p.K / p.groupsize;
+    if (G % 8 == 0 && (reinterpret_cast<uintptr_t>(p.scales) & 15) == 0 &&
+        (reinterpret_cast<uintptr_t>(p.zeros) & 15) == 0) {
+      p.sz_tma = 1;
+      spb = 8 / (gemm::kBK / p.groupsize);
+    }
+  }
   // split K over a cluster of S CTAs (one CTA per SM): pick S so that the
-  // rounds of CTAs times the k-blocks per CTA (plus a fixed cost of about two
-  // blocks for filling and draining the pipeline) is smallest
+  // rounds of CTAs times the k-blocks per CTA plus a fixed cost per CTA is
+  // smallest (the pipeline fill, about 4 us on B200, is worth ~16 k-blocks)
   int S = 1, kbps = KB;
   long best = -1;
   for (int s = 1; s <= 8 && s <= KB; ++s) {
-    const int bps = (KB + s - 1) / s;
+    int bps = (KB + s - 1) / s;
+    if (s > 1) bps = (bps + spb - 1) / spb * spb;
     const int s_eff = (KB + bps - 1) / bps;
     const long rounds = (long(tiles) * s_eff + sm_count - 1) / sm_count;
-    const long cost = rounds * (bps + 2);
+    const long cost = rounds * (bps + 16);
     if (best < 0 || cost < best) {
       best = cost;
       S = s_eff;
@@ -574,9 +646,9 @@ static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int 
   p.splits = S;
   p.kb_per_split = kbps;
   p.tmem_cols = 512;  // A tiles (4 x 64 columns) + accumulators (<= 256 columns)
-  const size_t small = 1024 + size_t(2 * L::kNumW + L::kNumA + 4 + gemm::kXsSlots + gemm::kIssuers) * 8 + 64 +
-                       size_t(gemm::kXsSlots * 4 * MV) * 4;
-  const size_t smem = L::kRingBytes + small;
+  const size_t small = 1024 + size_t(2 * L::kNumW + L::kNumA + 4 + gemm::kXsSlots + gemm::kIssuers + 2 * gemm::kSzSlots) * 8 +
+                       64 + size_t(gemm::kXsSlots * 4 * MV) * 4;
+  const size_t smem = L::kRingBytes + L::kSzBytes + small;
   static_assert(L::kRingBytes >= (3 * 128 * MV + 128 * (MV < 4 ? 4 : MV)) * 4,
                 "reduction buffers must fit the idle ring");
 
@@ -594,6 +666,11 @@ static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int 
     e = make_tmap_2d(&p.tm_w, w, 2, uint64_t(p.K), p.N, uint64_t(p.K) * 2, 64, gemm::kBM, 128);
   }
   if (e == cudaSuccess) e = make_tmap_2d(&p.tm_x, p.x, 2, uint64_t(p.K), p.M, uint64_t(p.K) * 2, 64, MPAD, 128);
+  if (e == cudaSuccess && p.sz_tma) {
+    const uint64_t G = uint64_t(p.K / p.groupsize);
+    e = make_tmap_2d(&p.tm_s, p.scales, 2, G, p.N, G * 2, 8, gemm::kBM, 0);
+    if (e == cudaSuccess) e = make_tmap_2d(&p.tm_z, p.zeros, 2, G, p.N, G * 2, 8, gemm::kBM, 0);
+  }
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gemm::wq_gemm_kernel<FMT, MPAD, MV>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;

@@ -62,21 +62,33 @@ struct GemvFmt<WQ_BF16> {
   static constexpr int kRowBytes = 512;
 };
 
-constexpr int kRB = 32;                 // rows per stage (one per producer lane)
-constexpr int kConsumerWarps = 8;
-// M <= 2: a producer warp keeps the ring full ahead of the eight consumer warps
-// (two CTAs per SM at M = 1, one at M = 2).  M >= 3 (the activations of a chunk
-// need more registers): one CTA per SM of eight consumer warps and no producer,
-// so each thread may hold up to 255 registers; the last warp to finish a stage
-// refills its slot.
-__host__ __device__ constexpr bool gemv_has_producer(int mm) { return mm <= 2; }
-__host__ __device__ constexpr int gemv_ctas_per_sm(int mm) { return mm <= 1 ? 2 : 1; }
-__host__ __device__ constexpr int gemv_threads(int mm) { return 32 * (kConsumerWarps + (gemv_has_producer(mm) ? 1 : 0)); }
+constexpr int kJ = 4;  // rows of a stage each consumer warp takes
+// Launch shape per format and M (measured on B200):
+//  * M = 1, int4 / int8 / bf16: two CTAs per SM, each with eight consumer warps
+//    and a producer warp that keeps the ring full; the next layer's CTAs can
+//    start while the last CTAs of this one drain (programmatic dependent launch);
+//  * M = 1, FP6 (decode-bound): one CTA per SM with sixteen consumer warps and a
+//    producer, so every SM carries the same share;
+//  * M = 2: one CTA per SM, eight consumer warps and a producer (168 registers a
+//    thread);
+//  * M >= 3: one CTA per SM, eight consumer warps and no producer, so each thread
+//    may hold up to 255 registers (the activations of a chunk need them); the
+//    last warp to finish a stage refills its slot.
+// A stage holds kJ rows per consumer warp.
+__host__ __device__ constexpr bool gemv_has_producer(int, int mm) { return mm <= 2; }
+__host__ __device__ constexpr int gemv_cw(int fmt, int mm) { return (mm == 1 && fmt == WQ_FP6_E3M2) ? 16 : 8; }
+__host__ __device__ constexpr int gemv_rb(int fmt, int mm) { return kJ * gemv_cw(fmt, mm); }
+__host__ __device__ constexpr int gemv_ctas_per_sm(int fmt, int mm) { return (mm == 1 && fmt != WQ_FP6_E3M2) ? 2 : 1; }
+__host__ __device__ constexpr int gemv_threads(int fmt, int mm) {
+  return 32 * (gemv_cw(fmt, mm) + (gemv_has_producer(fmt, mm) ? 1 : 0));
+}
+__host__ __device__ constexpr bool gemv_lane_partials(int mm) { return mm <= 2; }
 
 template <int FMT, int MM>
 struct GemvLayout {
   static constexpr int kChunkK = 32 * GemvFmt<FMT>::kLaneK;
   static constexpr int kXBytes = kChunkK * 2;  // one chunk of one activation row
+  static constexpr int kRB = gemv_rb(FMT, MM);  // rows per stage
   static constexpr int kStageBytes = (kRB * GemvFmt<FMT>::kRowBytes + MM * kXBytes + 127) / 128 * 128;
 };
 
@@ -262,11 +274,13 @@ __device__ __forceinline__ void advance(StagePos& p, int NS, int NRB, int C) {
 }
 
 template <int FMT, int MM>
-__global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_kernel(const __grid_constant__ GemvParams a) {
+__global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, MM)) gemv_kernel(const __grid_constant__ GemvParams a) {
   using F = GemvFmt<FMT>;
   using L = GemvLayout<FMT, MM>;
   constexpr int kChunkK = L::kChunkK;
-  constexpr bool kProducer = gemv_has_producer(MM);
+  constexpr bool kProducer = gemv_has_producer(FMT, MM);
+  constexpr int CWN = gemv_cw(FMT, MM);
+  constexpr int kRB = L::kRB;
   extern __shared__ __align__(1024) uint8_t smem[];
 
   const int NS = a.stages;
@@ -275,7 +289,12 @@ __global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_k
   uint64_t* empty = full + NS;                          // [NS] warps finished reading the slot's stage
   int* done_cnt = reinterpret_cast<int*>(empty + NS);  // [NS] arrivals counted, to elect the refilling warp
   int* last_issued = done_cnt + NS;                    // [NS] stage last issued into the slot
-  float* part = reinterpret_cast<float*>(last_issued + NS + (NS & 1));  // [C][R][MM], 8-byte aligned
+  // partial sums.  Lane partials (M <= 2): [R][MM][32 lanes], each (row, lane)
+  // entry owned by one thread, so stages add into it with no cross-lane step and
+  // the lanes are summed once in the epilogue.  Otherwise [C][R][MM]: one value
+  // per chunk after a shuffle reduction.
+  constexpr bool kLanePart = gemv_lane_partials(MM);
+  float* part = reinterpret_cast<float*>(last_issued + NS + (NS & 1));
   const int C = (a.K + kChunkK - 1) / kChunkK;
   const int n0 = blockIdx.x * a.rows_per_cta;
   const int R = min(a.rows_per_cta, a.N - n0);
@@ -318,10 +337,12 @@ __global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_k
 
   if (a.pdl) pdl_launch_dependents();
   const int T0 = min(T, NS);
+  if constexpr (kLanePart)
+    for (int i = threadIdx.x; i < R * MM * 32; i += blockDim.x) part[i] = 0.f;
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], CWN);
       done_cnt[s] = 0;
       last_issued[s] = -1;
     }
@@ -382,23 +403,26 @@ __global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_k
     int cur_c = -1;
     XRegs<FMT, MM> xr;
     const DecodeConsts<FMT> dc = make_decode_consts<FMT>();
-    constexpr int J = kRB / kConsumerWarps;  // rows of a stage this warp takes (4)
+    constexpr int J = kJ;
     const int gshift = (FMT == WQ_INT4) ? __ffs(a.groupsize) - 1 : 0;
     const int G = (FMT == WQ_INT4) ? (a.K >> gshift) : 0;
     // int4: raw 16-bit scale and zero of this warp's rows at the lane's group,
     // fetched one stage ahead into the other of two register sets; the load
     // zero-extends, so no instruction touches them before the fold a stage later
+    // (rows past N are skipped: only the last CTA has them)
+    const int G8 = G * CWN;
     auto fetch_sz = [&](const StagePos& p, uint32_t (&ds)[J], uint32_t (&dz)[J]) {
       if constexpr (FMT == WQ_INT4) {
-        const int rows = min(kRB, R - p.rb * kRB);
         const int k0 = p.c * kChunkK + lane * F::kLaneK;
-        if (k0 >= a.K) return;
-        const size_t off = size_t(n0 + p.rb * kRB + cw) * G + (k0 >> gshift);
+        const int row = n0 + p.rb * kRB + cw;
+        const int off = row * G + (k0 >> gshift);
+        const uint16_t* sp = a.scales + off;
+        const uint16_t* zp = a.zeros + off;
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-          if (cw + j * kConsumerWarps < rows) {
-            ds[j] = ld_nc_u16_u32(a.scales + off + size_t(j * kConsumerWarps) * G);
-            dz[j] = ld_nc_u16_u32(a.zeros + off + size_t(j * kConsumerWarps) * G);
+          if (k0 < a.K && row + j * CWN < a.N) {
+            ds[j] = ld_nc_u16_u32(sp + j * G8);
+            dz[j] = ld_nc_u16_u32(zp + j * G8);
           }
         }
       }
@@ -413,32 +437,28 @@ __global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_k
       if (has_next) fetch_sz(nx, ss_next, zz_next);
       if (!mbar_wait(&full[p.slot], p.phase)) return false;
       const int rows = min(kRB, R - p.rb * kRB);
-      const uint8_t* st = ring + size_t(p.slot) * L::kStageBytes;
+      const uint8_t* st = ring + p.slot * L::kStageBytes;
       if (p.c != cur_c) {
         load_x_smem<FMT, MM>(xr, st + kRB * F::kRowBytes, lane, p.c * kChunkK + lane * F::kLaneK < a.K);
         cur_c = p.c;
       }
-      // all J rows of this warp at once: independent chains interleave (the row
-      // test is uniform across the warp)
+      // all J rows of this warp at once: independent chains interleave.  Rows
+      // past the stage's last box hold stale shared memory; they are computed
+      // all the same (no branch) and never stored.
       float acc[J][MM];
 #pragma unroll
       for (int j = 0; j < J; ++j) {
-        const int i = cw + j * kConsumerWarps;
-        if (i < rows) {
-          if constexpr (FMT == WQ_FP6_E3M2)
-            lane_dot<FMT, MM>(st + i * 512, st + kRB * 512 + i * 256, lane, xr, dc, acc[j]);
-          else
-            lane_dot<FMT, MM>(st + i * F::kRowBytes, nullptr, lane, xr, dc, acc[j]);
-          if constexpr (FMT == WQ_INT4) {
-            // sum over the lane's 32 k (one group): s * sum(q x) + z * sum(x)
-            const float sc = __uint_as_float(ss[j] << 16);
-            const float zc = __uint_as_float(zz[j] << 16);
+        const int i = cw + j * CWN;
+        if constexpr (FMT == WQ_FP6_E3M2)
+          lane_dot<FMT, MM>(st + i * 512, st + kRB * 512 + i * 256, lane, xr, dc, acc[j]);
+        else
+          lane_dot<FMT, MM>(st + i * F::kRowBytes, nullptr, lane, xr, dc, acc[j]);
+        if constexpr (FMT == WQ_INT4) {
+          // sum over the lane's 32 k (one group): s * sum(q x) + z * sum(x)
+          const float sc = __uint_as_float(ss[j] << 16);
+          const float zc = __uint_as_float(zz[j] << 16);
 #pragma unroll
-            for (int m = 0; m < MM; ++m) acc[j][m] = fmaf(sc, acc[j][m], zc * xr.xsum[m]);
-          }
-        } else {
-#pragma unroll
-          for (int m = 0; m < MM; ++m) acc[j][m] = 0.f;
+          for (int m = 0; m < MM; ++m) acc[j][m] = fmaf(sc, acc[j][m], zc * xr.xsum[m]);
         }
       }
       // every lane's shared-memory reads of the stage are done: release them on
@@ -450,7 +470,7 @@ __global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_k
         if constexpr (!kProducer) {
           // the counter elects the last warp, which waits for the barrier
           // (acquiring every warp's reads) and refills the slot with stage t + NS
-          if (atomicAdd(&done_cnt[p.slot], 1) == kConsumerWarps - 1) {
+          if (atomicAdd(&done_cnt[p.slot], 1) == CWN - 1) {
             done_cnt[p.slot] = 0;
             ok = mbar_wait(&empty[p.slot], p.phase);
             if (ok && t + NS < T) {
@@ -463,25 +483,39 @@ __global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_k
         }
       }
       if (!kProducer && !__shfl_sync(0xFFFFFFFFu, int(ok), 0)) return false;
-      // transposed butterfly: 6 shuffles reduce the 4 rows; lane 8j holds row j
-      static_assert(J == 4, "reduction below assumes 4 rows per warp and stage");
+      if constexpr (kLanePart) {
+        // add the lane partials of the warp's rows (rows past R belong to the
+        // next CTA or hold stale data: skipped, uniformly across the warp)
 #pragma unroll
-      for (int m = 0; m < MM; ++m) {
-        const bool hi16 = lane & 16;
-        float k0v = hi16 ? acc[2][m] : acc[0][m];
-        float k1v = hi16 ? acc[3][m] : acc[1][m];
-        k0v += __shfl_xor_sync(0xFFFFFFFFu, hi16 ? acc[0][m] : acc[2][m], 16);
-        k1v += __shfl_xor_sync(0xFFFFFFFFu, hi16 ? acc[1][m] : acc[3][m], 16);
-        const bool hi8 = lane & 8;
-        float kv = hi8 ? k1v : k0v;
-        kv += __shfl_xor_sync(0xFFFFFFFFu, hi8 ? k0v : k1v, 8);
-        kv += __shfl_xor_sync(0xFFFFFFFFu, kv, 4);
-        kv += __shfl_xor_sync(0xFFFFFFFFu, kv, 2);
-        kv += __shfl_xor_sync(0xFFFFFFFFu, kv, 1);
-        if ((lane & 7) == 0) {
-          const int j = lane >> 3;  // 2 * (bit 4) + (bit 3)
-          const int i = cw + j * kConsumerWarps;
-          if (i < rows) part[(size_t(p.c) * R + p.rb * kRB + i) * MM + m] = kv;
+        for (int j = 0; j < J; ++j) {
+          const int row = p.rb * kRB + cw + j * CWN;
+          if (row < R) {
+            float* dst = part + row * (MM * 32) + lane;
+#pragma unroll
+            for (int m = 0; m < MM; ++m) dst[m * 32] += acc[j][m];
+          }
+        }
+      } else {
+        // transposed butterfly: 6 shuffles reduce the 4 rows; lane 8j holds row j
+        static_assert(J == 4, "reduction below assumes 4 rows per warp and stage");
+#pragma unroll
+        for (int m = 0; m < MM; ++m) {
+          const bool hi16 = lane & 16;
+          float k0v = hi16 ? acc[2][m] : acc[0][m];
+          float k1v = hi16 ? acc[3][m] : acc[1][m];
+          k0v += __shfl_xor_sync(0xFFFFFFFFu, hi16 ? acc[0][m] : acc[2][m], 16);
+          k1v += __shfl_xor_sync(0xFFFFFFFFu, hi16 ? acc[1][m] : acc[3][m], 16);
+          const bool hi8 = lane & 8;
+          float kv = hi8 ? k1v : k0v;
+          kv += __shfl_xor_sync(0xFFFFFFFFu, hi8 ? k0v : k1v, 8);
+          kv += __shfl_xor_sync(0xFFFFFFFFu, kv, 4);
+          kv += __shfl_xor_sync(0xFFFFFFFFu, kv, 2);
+          kv += __shfl_xor_sync(0xFFFFFFFFu, kv, 1);
+          if ((lane & 7) == 0) {
+            const int j = lane >> 3;  // 2 * (bit 4) + (bit 3)
+            const int i = cw + j * CWN;
+            if (i < rows) part[((p.c * R) + p.rb * kRB + i) * MM + m] = kv;
+          }
         }
       }
       p = nx;
@@ -519,11 +553,22 @@ __global__ void __launch_bounds__(gemv_threads(MM), gemv_ctas_per_sm(MM)) gemv_k
     }
     return;
   }
+  // sum the partials of each (row, activation row) in a fixed order: the 32 lane
+  // partials (starting at a rotating lane so that neighbouring threads read
+  // different banks), or the per-chunk values in chunk order
   for (int idx = threadIdx.x; idx < R * MM; idx += blockDim.x) {
-    const int m = idx / R;
-    const int r = idx - m * R;
+    int r, m;
     float v = 0.f;
-    for (int c = 0; c < C; ++c) v += part[(size_t(c) * R + r) * MM + m];
+    if constexpr (kLanePart) {
+      r = idx / MM;
+      m = idx - r * MM;
+      const float* src = part + idx * 32;
+      for (int l = 0; l < 32; ++l) v += src[(l + idx) & 31];
+    } else {
+      m = idx / R;
+      r = idx - m * R;
+      for (int c = 0; c < C; ++c) v += part[(c * R + r) * MM + m];
+    }
     const int n = n0 + r;
     if constexpr (FMT == WQ_INT8) {
       v *= fp16_bits_to_float(a.scales[n]);
@@ -545,23 +590,24 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   using F = GemvFmt<FMT>;
   GemvParams p = p0;
   const int C = (p.K + L::kChunkK - 1) / L::kChunkK;
-  const int target = sm_count * gemv_ctas_per_sm(MM);
-  const size_t kGemvSmemBudget = kGemvSmemPerSm / gemv_ctas_per_sm(MM);
+  const int target = sm_count * gemv_ctas_per_sm(FMT, MM);
+  const size_t kGemvSmemBudget = kGemvSmemPerSm / gemv_ctas_per_sm(FMT, MM);
   // rows per CTA: a multiple of the box height, about N / target
   int R = (p.N + target * kBoxRows - 1) / (target * kBoxRows) * kBoxRows;
-  // keep the partial-sum area within a quarter of the budget
-  const int max_r = int((kGemvSmemBudget / 4) / (size_t(C) * MM * 4)) / kBoxRows * kBoxRows;
+  // keep the partial-sum area within half (lane partials) or a quarter of the budget
+  const size_t part_row = gemv_lane_partials(MM) ? size_t(32) * MM * 4 : size_t(C) * MM * 4;
+  const int max_r = int((gemv_lane_partials(MM) ? kGemvSmemBudget / 2 : kGemvSmemBudget / 4) / part_row) / kBoxRows * kBoxRows;
   if (R > max_r) R = max_r;
   if (R < kBoxRows) R = kBoxRows;
   p.rows_per_cta = R;
   p.box_rows = kBoxRows;
-  const size_t fixed = 8 * 24 + 16 + size_t(C) * R * MM * 4;
+  const size_t fixed = 8 * 24 + 16 + size_t(R) * part_row;
   if (fixed + 2 * size_t(L::kStageBytes) > 200 * 1024) return cudaErrorInvalidValue;
   int stages = fixed < kGemvSmemBudget ? int((kGemvSmemBudget - fixed) / L::kStageBytes) : 2;
   if (stages > 8) stages = 8;
   if (stages < 2) stages = 2;
   p.stages = stages;
-  const size_t smem = size_t(stages) * L::kStageBytes + size_t(stages) * 24 + 16 + size_t(C) * R * MM * 4;
+  const size_t smem = size_t(stages) * L::kStageBytes + size_t(stages) * 24 + 16 + size_t(R) * part_row;
 
   // tensor maps: rows of packed bytes viewed as 32-bit elements, one chunk per box
   cudaError_t e;
@@ -581,7 +627,7 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   const int grid = (p.N + R - 1) / R;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(gemv_threads(MM));
+  cfg.blockDim = dim3(gemv_threads(FMT, MM));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -20,6 +20,8 @@ cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uin
 struct GemmParams {
   CUtensorMap tm_w;        // packed weights (FP6: the 4-bit plane; bf16: W)
   CUtensorMap tm_w2;       // FP6: the 2-bit plane
+  CUtensorMap tm_s;        // int4 with sz_tma: scales [N, K/g] bf16, boxes of 8 groups x 128 rows
+  CUtensorMap tm_z;        // int4 with sz_tma: zeros, same boxes
   CUtensorMap tm_x;        // activations, 128-byte swizzled boxes
   const uint16_t* x;
   const void* packed;
@@ -30,6 +32,7 @@ struct GemmParams {
   int splits;              // CTAs of a cluster splitting K (set by the launcher)
   int kb_per_split;        // 128-wide k-blocks per split (set by the launcher)
   uint32_t tmem_cols;      // tensor-memory columns allocated per CTA
+  int sz_tma;              // int4: scales / zeros staged by tensor copies (row pitch a multiple of 16 B)
   int pdl;
 };
 

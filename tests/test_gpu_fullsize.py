@@ -1,0 +1,95 @@
+"""GPU parity at the benchmarked layer sizes, in the benchmark's launch setup.
+
+Every layer shape of the benchmark configurations appears here at full size
+(Llama-2-7B int4 g32 / g128 at M = 1, Llama-70B FP6 at M = 1..16, OPT-30B
+int8 / int4-g128 / FP6 / bf16 at M up to 32, the 4096 x 4096 int8 layer).  The
+product side quantizes and packs the whole weight with libwq and runs the layer
+the way bench.py does: launched with programmatic dependent launch inside a CUDA
+graph, after another layer in the same graph.  The oracle regenerates only a
+sample of weight rows (the seeded generator draws each 1024-row block on its
+own), quantizes them itself and computes those outputs over the full K in fp64;
+the sampled columns of y must meet the tolerance.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import gemm_wq_linear_b200 as wq
+import workloads
+from oracle import linear
+from wq_cases import compare, oracle_weights, x_bits
+
+pytestmark = pytest.mark.gpu
+
+# (fmt, groupsize, K, N, M)
+CASES = [
+    ("int4", 32, 4096, 22016, 1),
+    ("int4", 128, 11008, 4096, 1),
+    ("int4", 32, 4096, 12288, 1),
+    ("int4", 128, 7168, 28672, 8),
+    ("int4", 128, 28672, 7168, 32),
+    ("fp6", 0, 8192, 57344, 1),
+    ("fp6", 0, 28672, 8192, 4),
+    ("fp6", 0, 8192, 10240, 16),
+    ("int8", 0, 4096, 4096, 1),
+    ("int8", 0, 7168, 28672, 2),
+    ("int8", 0, 7168, 21504, 32),
+    ("bf16", 0, 7168, 7168, 1),
+    ("bf16", 0, 28672, 7168, 16),
+]
+
+SAMPLE_ROWS = 192
+
+
+def _sample_rows(N, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(N, size=min(N, SAMPLE_ROWS - 4), replace=False).tolist())
+    rows.update({0, 1, N - 2, N - 1})  # first and last rows (tail of the last CTA / tile)
+    return np.array(sorted(rows))
+
+
+def _run_like_bench(x, pw, M, N):
+    """A warm-up layer then the layer under test, both PDL launches captured in
+    one CUDA graph, replayed twice (the second replay's y is compared)."""
+    stream = torch.cuda.Stream()
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    y_pre = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    with torch.cuda.stream(stream):
+        wq.linear(x, pw, out=y_pre, stream=stream, flags=wq.WQ_LAUNCH_PDL)
+        wq.linear(x, pw, out=y, stream=stream, flags=wq.WQ_LAUNCH_PDL)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        wq.linear(x, pw, out=y_pre, stream=stream, flags=wq.WQ_LAUNCH_PDL)
+        wq.linear(x, pw, out=y, stream=stream, flags=wq.WQ_LAUNCH_PDL)
+    y.fill_(float("nan"))
+    graph.replay()
+    graph.replay()
+    torch.cuda.synchronize()
+    wq.wq_sync_status()
+    assert torch.equal(y, y_pre)
+    return y.cpu()
+
+
+@pytest.mark.parametrize("fmt,g,K,N,M", CASES, ids=[f"{c[0]}-g{c[1]}-K{c[2]}-N{c[3]}-M{c[4]}" for c in CASES])
+def test_full_size_sampled_rows(fmt, g, K, N, M):
+    seed = 4000 + K % 997 + N % 991 + M
+    W = workloads.weights(N, K, seed)
+    pw = wq.PackedWeight.quantize(W, fmt, g)
+    del W
+    x = workloads.activations(M, K, seed + 1)
+    y = _run_like_bench(x.cuda(), pw, M, N)
+
+    rows = _sample_rows(N, seed)
+    blocks = {}
+    Wd = np.empty((len(rows), K), dtype=np.float64)
+    for i, r in enumerate(rows):
+        b = int(r) // 1024
+        if b not in blocks:
+            r0 = b * 1024
+            blocks[b] = (r0, workloads.weights(N, K, seed, rows=slice(r0, min(N, r0 + 1024))).numpy())
+        r0, Wb = blocks[b]
+        Wd[i] = oracle_weights(fmt, Wb[int(r) - r0:int(r) - r0 + 1], g)[0]
+    y_ref = linear.linear_ref(x_bits(x), Wd)  # [M, len(rows)]
+    compare(y[:, rows], y_ref)

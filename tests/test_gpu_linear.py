@@ -145,3 +145,17 @@ def test_linear_zero_weight_rows():
 
 def test_sync_status_ok():
     wq.wq_sync_status()
+
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+@pytest.mark.parametrize("M", [5, 8, 16, 32])
+def test_linear_int4_gemm_staged_scales(g, M):
+    """K = 2048: the scale rows are a multiple of 16 bytes, so the tensor-core
+    kernel stages scales and zeros with tensor copies (8-group boxes spanning
+    several k-blocks, splits aligned to them); N = 700 leaves a ragged last tile."""
+    N, K = 700, 2048
+    W = workloads.weights(N, K, seed=600 + g)
+    pw = product_weight("int4", W, g)
+    x = workloads.activations(M, K, seed=700 + M)
+    y = gpu_linear(x, pw)
+    compare(y, linear.linear_ref(x_bits(x), oracle_weights("int4", W.numpy(), g)))
