@@ -262,10 +262,11 @@ struct StagePos {
   int rb;
   int c;
 };
-__device__ __forceinline__ void advance(StagePos& p, int NS, int NRB, int C) {
+// chunks cycle through [clo, chi), the CTA's share of K
+__device__ __forceinline__ void advance(StagePos& p, int NS, int NRB, int clo, int chi) {
   if (++p.rb == NRB) {
     p.rb = 0;
-    p.c = (p.c + 1 == C) ? 0 : p.c + 1;
+    p.c = (p.c + 1 == chi) ? clo : p.c + 1;
   }
   if (++p.slot == NS) {
     p.slot = 0;
@@ -296,13 +297,19 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
   constexpr bool kLanePart = gemv_lane_partials(MM);
   float* part = reinterpret_cast<float*>(last_issued + NS + (NS & 1));
   const int C = (a.K + kChunkK - 1) / kChunkK;
-  const int n0 = blockIdx.x * a.rows_per_cta;
+  // split K: the S CTAs of a cluster share a row block, rank q taking chunks
+  // [CLO, CHI); rank 0 sums the cluster's partials at the end
+  const int S = a.ksplit;
+  const int rank = blockIdx.x % S;
+  const int n0 = (blockIdx.x / S) * a.rows_per_cta;
   const int R = min(a.rows_per_cta, a.N - n0);
   const int NRB = (R + kRB - 1) / kRB;
-  const int T = C * NRB;
+  const int CLO = rank * a.chunks_per_split;
+  const int CHI = min(C, CLO + a.chunks_per_split);
+  const int T = (CHI - CLO) * NRB;
   // each CTA starts at a different chunk so that concurrent CTAs fetch
   // different parts of x
-  const int c_rot = blockIdx.x % C;
+  const int c_rot = CLO + (blockIdx.x / S) % (CHI - CLO);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t policy = l2_policy_evict_first();
@@ -356,13 +363,13 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
       for (int t = 0; t < T0; ++t) {
         issue_w(q);
         last_issued[q.slot] = t;
-        advance(q, NS, NRB, C);
+        advance(q, NS, NRB, CLO, CHI);
       }
       if (a.pdl) pdl_wait();
       q = {0, 0u, 0, c_rot};
       for (int t = 0; t < T0; ++t) {
         issue_x(q);
-        advance(q, NS, NRB, C);
+        advance(q, NS, NRB, CLO, CHI);
       }
     }
   }
@@ -388,10 +395,10 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
           StagePos q = {0, 0u, 0, c_rot};
           for (int t2 = 0; t2 < T0; ++t2) {
             issue_x(q);
-            advance(q, NS, NRB, C);
+            advance(q, NS, NRB, CLO, CHI);
           }
         }
-        advance(p, NS, NRB, C);
+        advance(p, NS, NRB, CLO, CHI);
       }
       if (failed && a.pdl) pdl_wait();
     }
@@ -433,7 +440,7 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
     auto stage = [&](int t, StagePos& p, StagePos& pr, bool has_next, const uint32_t (&ss)[J],
                      const uint32_t (&zz)[J], uint32_t (&ss_next)[J], uint32_t (&zz_next)[J]) -> bool {
       StagePos nx = p;
-      advance(nx, NS, NRB, C);
+      advance(nx, NS, NRB, CLO, CHI);
       if (has_next) fetch_sz(nx, ss_next, zz_next);
       if (!mbar_wait(&full[p.slot], p.phase)) return false;
       const int rows = min(kRB, R - p.rb * kRB);
@@ -519,7 +526,7 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
         }
       }
       p = nx;
-      advance(pr, NS, NRB, C);
+      advance(pr, NS, NRB, CLO, CHI);
       return true;
     };
     uint32_t sA[J], zA[J], sB[J], zB[J];
@@ -527,7 +534,7 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
     for (int j = 0; j < J; ++j) sA[j] = zA[j] = sB[j] = zB[j] = 0u;
     StagePos p = {0, 0u, 0, c_rot};
     StagePos pr = p;  // position of stage t + NS
-    for (int i = 0; i < NS; ++i) advance(pr, NS, NRB, C);
+    for (int i = 0; i < NS; ++i) advance(pr, NS, NRB, CLO, CHI);
     fetch_sz(p, sA, zA);
     for (int t = 0; t < T; t += 2) {
       if (!stage(t, p, pr, t + 1 < T, sA, zA, sB, zB)) {
@@ -544,15 +551,42 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
   // ---------------------------------------------------------------- epilogue
   const bool any_failed = __syncthreads_or(failed);
   if (any_failed) {
-    // wait (bounded) until every copy issued into the ring has landed, then leave
+    // wait (bounded) until every copy issued into the ring has landed
     if (threadIdx.x == 0) {
       for (int s = 0; s < NS; ++s) {
         const int u = last_issued[s];
         if (u >= 0) mbar_wait(&full[s], (u / NS) & 1);
       }
     }
-    return;
   }
+  if constexpr (kLanePart) {
+    if (S > 1) {
+      // every CTA of the cluster reaches both cluster barriers, failed or not
+      cluster_sync_all();  // all lane partials of the cluster are final
+      if (rank == 0 && !any_failed) {
+        for (int idx = threadIdx.x; idx < R * MM; idx += blockDim.x) {
+          const int r = idx / MM;
+          const int m = idx - r * MM;
+          const uint32_t base = smem_u32(part + idx * 32);
+          float v = 0.f;
+          for (int q = 0; q < S; ++q) {
+            const uint32_t src = q == 0 ? base : map_to_rank(base, uint32_t(q));
+            for (int l = 0; l < 32; ++l) v += ld_cluster_f32(src + 4 * ((l + idx) & 31));
+          }
+          const int n = n0 + r;
+          if constexpr (FMT == WQ_INT8) {
+            v *= fp16_bits_to_float(a.scales[n]);
+          } else if constexpr (FMT == WQ_FP6_E3M2) {
+            v = (v * 0x1p124f) * fp16_bits_to_float(a.scales[n]);
+          }
+          a.y[size_t(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        }
+      }
+      cluster_sync_all();  // keep every CTA's shared memory until rank 0 has read it
+      return;
+    }
+  }
+  if (any_failed) return;
   // sum the partials of each (row, activation row) in a fixed order: the 32 lane
   // partials (starting at a rotating lane so that neighbouring threads read
   // different banks), or the per-chunk values in chunk order
@@ -599,6 +633,22 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   const int max_r = int((gemv_lane_partials(MM) ? kGemvSmemBudget / 2 : kGemvSmemBudget / 4) / part_row) / kBoxRows * kBoxRows;
   if (R > max_r) R = max_r;
   if (R < kBoxRows) R = kBoxRows;
+  // split K over a cluster when the rows per CTA would not fill one stage (small
+  // N): each CTA then takes one full stage of rows and a share of the chunks
+  int S = 1, CPS = C;
+  if (gemv_lane_partials(MM) && R < L::kRB) {
+    const int nblk = (p.N + L::kRB - 1) / L::kRB;
+    int s = target / nblk;
+    s = s > 8 ? 8 : s;
+    s = s > C ? C : s;
+    if (s >= 2) {
+      CPS = (C + s - 1) / s;
+      S = (C + CPS - 1) / CPS;
+      R = L::kRB;
+    }
+  }
+  p.ksplit = S;
+  p.chunks_per_split = CPS;
   p.rows_per_cta = R;
   p.box_rows = kBoxRows;
   const size_t fixed = 8 * 24 + 16 + size_t(R) * part_row;
@@ -624,17 +674,32 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gemv_kernel<FMT, MM>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  const int grid = (p.N + R - 1) / R;
+  const int grid = (p.N + R - 1) / R * S;
+  if (S > 1) {
+    e = cudaFuncSetAttribute(gemv_kernel<FMT, MM>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(gemv_threads(FMT, MM));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (S > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = S;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (p.pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = p.pdl ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, gemv_kernel<FMT, MM>, p);
 }
 

@@ -50,6 +50,8 @@ struct GemvParams {
   uint16_t* y;             // bf16 [M, N]
   int M, N, K, groupsize, fmt;
   int rows_per_cta;        // set by the launcher
+  int ksplit;              // CTAs of a cluster splitting K (lane-partial path only), set by the launcher
+  int chunks_per_split;    // K-chunks per split, set by the launcher
   int stages;              // shared-memory ring depth, set by the launcher
   int box_rows;            // rows per tensor-copy box (rows_per_cta is a multiple)
   int pdl;                 // programmatic dependent launch enabled

@@ -144,8 +144,10 @@ wq_status wq_prepack_fp6(const uint8_t* code, int64_t N, int64_t K, void* packed
  *   zeros:  device bf16 [N, K/g] for WQ_INT4, must be NULL otherwise
  *   y:      device bf16 [M, N], written with round-to-nearest-even
  * M in [0, 32].  Dispatch: M <= 4 runs the CUDA-core split-K GEMV; larger M runs
- * the tensor-core (tcgen05) swap-AB GEMM where built.  Launch errors give
- * WQ_ERR_CUDA.  Buffers must not overlap y. */
+ * the tensor-core (tcgen05) swap-AB GEMM.  For WQ_INT4 with (K / groupsize) a
+ * multiple of 8 and 16-byte aligned scales and zeros, the GEMM stages them with
+ * tensor copies; otherwise it reads them with ordinary loads (same result).
+ * Launch errors give WQ_ERR_CUDA.  Buffers must not overlap y. */
 wq_status wq_linear(const void* x, const void* packed, const void* scales, const void* zeros,
                     void* y, int64_t M, int64_t N, int64_t K, int fmt, int groupsize,
                     void* cuda_stream);

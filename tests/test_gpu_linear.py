@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 N_SMALL, K_SMALL = 700, 2176
 VARIANTS = [("int8", 0), ("int4", 32), ("int4", 64), ("int4", 128), ("fp6", 0), ("bf16", 0)]
-MS = [1, 2, 3, 4, 5, 8, 16, 32]
+MS = [1, 2, 3, 4, 5, 8, 9, 16, 32]
 
 _cache = {}
 
