@@ -181,8 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   uint64_t* full_w = bars;             // [NW]  tensor copies landed
   uint64_t* mdone = full_w + NW;       // [NW]  MMAs of the stage's block completed
   uint64_t* afull = mdone + NW;        // [NA]  A tile written to TMEM
-  uint64_t* dempty = afull + NA;       // [4]   int4: accumulator block-buffer folded
-  uint64_t* xready = dempty + 4;       // [kXsSlots] int4: group sums of x of a block written
+  uint64_t* dempty = afull + NA;       // [16]  int4: accumulator block-buffer folded
+  uint64_t* xready = dempty + 16;      // [kXsSlots] int4: group sums of x of a block written
   uint64_t* done = xready + kXsSlots;  // [kIssuers] every MMA of an issuer completed
   uint64_t* szfull = done + kIssuers;  // [kSzSlots] int4: scale / zero box landed
   uint64_t* szfree = szfull + kSzSlots;  // [kSzSlots] int4: every block of the box folded
@@ -206,8 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
   // TMEM columns: [0, NA * 64) A tiles, then accumulators (int4: ndb block-buffers
   // of gpb groups; otherwise one per issuer)
   constexpr uint32_t kDCol = NA * kACols;
-  const int ndb = kInt4 ? min(4, 256 / (gpb * MPAD)) : 1;
-  const int lag = ndb - 1;  // int4: block j is folded while block j + lag is dequantized
+  // int4 accumulator block-buffers (a power of two, up to 16 when the groups are
+  // wide): the MMAs of block j reuse the buffer of block j - ndb, so a deep ring
+  // keeps them from waiting on the fold
+  const int ndb = kInt4 ? min(16, 256 / (gpb * MPAD)) : 1;
+  const int lag = min(3, ndb - 1);  // int4: block j is folded while block j + lag is dequantized
   const uint32_t tmem_cols = a.tmem_cols;
 
   if (a.pdl) pdl_launch_dependents();
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
       mbar_init(&mdone[i], 1);
     }
     for (int i = 0; i < NA; ++i) mbar_init(&afull[i], kDqWarps);
-    for (int i = 0; i < 4; ++i) mbar_init(&dempty[i], 4);
+    for (int i = 0; i < 16; ++i) mbar_init(&dempty[i], 4);
     for (int i = 0; i < kXsSlots; ++i) mbar_init(&xready[i], kXsWarps);
     for (int i = 0; i < kIssuers; ++i) mbar_init(&done[i], 1);
     for (int i = 0; i < kSzSlots; ++i) {
@@ -624,7 +627,7 @@ static cudaError_t launch_gemm_t(const GemmParams& p0, cudaStream_t stream, int 
   p.splits = S;
   p.kb_per_split = kbps;
   p.tmem_cols = 512;  // A tiles (4 x 64 columns) + accumulators (<= 256 columns)
-  const size_t small = 1024 + size_t(2 * L::kNumW + L::kNumA + 4 + gemm::kXsSlots + gemm::kIssuers + 2 * gemm::kSzSlots) * 8 +
+  const size_t small = 1024 + size_t(2 * L::kNumW + L::kNumA + 16 + gemm::kXsSlots + gemm::kIssuers + 2 * gemm::kSzSlots) * 8 +
                        64 + size_t(gemm::kXsSlots * 4 * MV) * 4;
   const size_t smem = L::kRingBytes + L::kSzBytes + small;
   static_assert(L::kRingBytes >= (3 * 128 * MV + 128 * (MV < 4 ? 4 : MV)) * 4,

@@ -450,12 +450,17 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
         cur_c = p.c;
       }
       // all J rows of this warp at once: independent chains interleave.  Rows
-      // past the stage's last box hold stale shared memory; they are computed
-      // all the same (no branch) and never stored.
+      // past the stage's last row are skipped (the test is uniform across the
+      // warp); their partials are zero and never stored.
       float acc[J][MM];
 #pragma unroll
       for (int j = 0; j < J; ++j) {
         const int i = cw + j * CWN;
+        if (i >= rows) {
+#pragma unroll
+          for (int m = 0; m < MM; ++m) acc[j][m] = 0.f;
+          continue;
+        }
         if constexpr (FMT == WQ_FP6_E3M2)
           lane_dot<FMT, MM>(st + i * 512, st + kRB * 512 + i * 256, lane, xr, dc, acc[j]);
         else
