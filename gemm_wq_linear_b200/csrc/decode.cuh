@@ -33,17 +33,6 @@ __device__ __forceinline__ uint32_t lop_and(uint32_t a, uint32_t b) {
 }
 __device__ __forceinline__ uint32_t rotl32(uint32_t x, int s) { return __funnelshift_l(x, x, s); }
 
-// (a0, a1) += (b0, b1): packed fp32 add of sm_100 (one instruction, two lanes).
-__device__ __forceinline__ void fadd2(float& a0, float& a1, float b0, float b1) {
-  asm("{.reg .b64 a, b;\n\t"
-      "mov.b64 a, {%0, %1};\n\t"
-      "mov.b64 b, {%2, %3};\n\t"
-      "add.rn.f32x2 a, a, b;\n\t"
-      "mov.b64 {%0, %1}, a;}\n"
-      : "+f"(a0), "+f"(a1)
-      : "f"(b0), "f"(b1));
-}
-
 // (a0, a1) += c, c a packed pair of fp32 constants held in a 64-bit register.
 __device__ __forceinline__ void fadd2c(float& a0, float& a1, uint64_t c) {
   asm("{.reg .b64 a;\n\t"
@@ -60,19 +49,6 @@ __device__ __forceinline__ uint64_t opaque_f32x2(float lo, float hi) {
   uint64_t r;
   asm volatile("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
   return r;
-}
-
-// (acc0, acc1) += (w0 * x0, w1 * x1): packed fp32 FMA of sm_100 (one
-// instruction for two lanes), each product rounded once into its accumulator.
-__device__ __forceinline__ void ffma2(float& acc0, float& acc1, float w0, float w1, float x0, float x1) {
-  asm("{.reg .b64 a, w, x;\n\t"
-      "mov.b64 a, {%0, %1};\n\t"
-      "mov.b64 w, {%2, %3};\n\t"
-      "mov.b64 x, {%4, %5};\n\t"
-      "fma.rn.f32x2 a, w, x, a;\n\t"
-      "mov.b64 {%0, %1}, a;}\n"
-      : "+f"(acc0), "+f"(acc1)
-      : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
 }
 
 // Packed fp32 pairs held as native 64-bit registers.
@@ -121,9 +97,6 @@ __device__ __forceinline__ void decode_int4_word(uint32_t w, uint32_t p[4]) {
   p[2] = lop_and_or(w >> 8, 0x000F000Fu, kBf16Magic128x2);
   p[3] = lop_and_or(w >> 12, 0x000F000Fu, kBf16Magic128x2);
 }
-
-// fp32 exponent field of 2^e.
-__host__ __device__ constexpr uint32_t f32_exp_bits(int e) { return uint32_t(127 + e) << 23; }
 
 // CUDA-core form, two words at a time.  wa, wb are two int4 words.  For nibble
 // n of both words, one LOP3 per word masks the nibble and ORs the exponent of

@@ -7,19 +7,22 @@
 // bandwidth bound: every generated token reads every weight once).  The kernel
 // reads each packed byte exactly once and hides dequantization under the stream:
 //
-//  * A CTA owns a contiguous block of R output rows over all of K (one
-//    contiguous region of the row-major packed matrix, so no cross-CTA
-//    reduction and a deterministic result).
+//  * A CTA owns a block of R output rows over its share of K.  When R would not
+//    fill one stage (small N), a thread-block cluster splits K and rank 0 sums
+//    the cluster's partials through distributed shared memory (no scratch, a
+//    fixed order: the result is deterministic).
 //  * K is cut into chunks of 32 lanes x LANE_K weights.  A stage of the
-//    shared-memory ring holds one chunk of up to 32 rows plus that chunk of x;
-//    warp 0 fills the ring with bulk asynchronous copies (TMA engine), one row
-//    per lane, completing on the stage's mbarrier, far ahead of the consumers.
-//  * Eight consumer warps take the rows of a stage; every lane reads its 16
-//    bytes (FP6: 16 + 8) of the row from shared memory, decodes them in
-//    registers (bit-parallel unpack, see decode.cuh) and multiplies with its
-//    activations held in registers for the whole chunk.  A shuffle butterfly
-//    reduces each (row, chunk); partials are summed in chunk order in shared
-//    memory, scaled and rounded to bf16.
+//    shared-memory ring holds one chunk of kJ rows per consumer warp plus, for
+//    a chunk's first stage, that chunk of x.  A producer warp (or, without one,
+//    the last consumer warp out of the stage) fills the ring with 2-D tensor
+//    copies of 8-row boxes and bulk copies of x, completing on the stage's
+//    mbarrier, far ahead of the consumers.
+//  * Each consumer lane reads its 16 bytes (FP6: 16 + 8) of a row from shared
+//    memory, decodes them in registers (explicit LOP3 / funnel-shift / PRMT PTX,
+//    decode.cuh) and multiplies with its activations, held in registers for the
+//    whole chunk, with the packed fp32 FMA.  Lane partials accumulate in shared
+//    memory across stages (M <= 2) or are reduced with shuffles per stage
+//    (M >= 3); the sums are scaled and rounded to bf16 once.
 //
 // Dequantization arithmetic (fp32 accumulation):
 //  * int4: decoded value q * 2^(p - 8) against activations scaled by 2^(8 - p)
