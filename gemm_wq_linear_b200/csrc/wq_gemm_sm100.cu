@@ -51,7 +51,7 @@ constexpr int kDqWarps = 16;  // dequant / epilogue warps: 4 per TMEM lane quadr
 constexpr int kDq0 = 1 + kIssuers;                    // first dequant warp
 constexpr int kThreads = 32 * (kDq0 + kDqWarps);      // + producer warp
 constexpr int kACols = kBK / 2;  // TMEM columns of one A tile (two bf16 per column)
-constexpr int kXsSlots = 32;     // int4: ring of per-block group sums of x
+constexpr int kXsSlots = 8;      // int4: ring of per-block group sums of x
 constexpr int kSzSlots = 8;      // int4: ring of staged scale / zero boxes
 
 template <int FMT>
@@ -383,92 +383,66 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
       }
     };
     // int4: fold the group accumulators of block j into acc (warps with u == j % 4)
-    // int4: fold the group accumulators of nb blocks j0, j0 + 4, ... (all of this
-    // warp group's, u == j0 % 4) into acc.  Every tensor-memory read of the batch
-    // is in flight before one wait: a wait costs a round trip behind the MMAs
-    // in flight, so deep accumulator rings fold several blocks per wait.
-    constexpr int LD = MV <= 8 ? 8 : MV;  // columns loaded per group
-    constexpr int kLoads = 32 / LD > 4 ? 4 : (32 / LD < 1 ? 1 : 32 / LD);  // group reads per wait
-    auto fold_blocks = [&](int j0, int nb) -> bool {
+    auto fold_block = [&](int j) -> bool {
       if constexpr (kInt4) {
+        const int db = j & (ndb - 1);
+        if (!mbar_wait(&mdone[j % NW], (j / NW) & 1) || !mbar_wait(&xready[j % kXsSlots], (j / kXsSlots) & 1))
+          return false;
         const int spb = 8 / gpb;
-        float scv[kLoads], zcv[kLoads];
-        uint32_t dv[kLoads][LD];
-        int n = 0;
-        for (int b = 0; b < nb; ++b) {
-          const int j = j0 + 4 * b;
-          if (!mbar_wait(&mdone[j % NW], (j / NW) & 1) || !mbar_wait(&xready[j % kXsSlots], (j / kXsSlots) & 1))
-            return false;
-          if (a.sz_tma) {
-            const int box = j / spb;
-            const int zs = box % kSzSlots;
-            if (!mbar_wait(&szfull[zs], (box / kSzSlots) & 1)) return false;
+        const int box = j / spb;
+        const int zs = box % kSzSlots;
+        if (a.sz_tma) {
+          // this row's scales and zeros of the block, from the staged box
+          if (!mbar_wait(&szfull[zs], (box / kSzSlots) & 1)) return false;
+          const uint16_t* sp = reinterpret_cast<const uint16_t*>(szring + zs * L::kSzSlotBytes) + r * 8 + (j % spb) * gpb;
+          const uint16_t* zp = sp + L::kSzSlotBytes / 4;
+#pragma unroll
+          for (int gi = 0; gi < 4; ++gi) {
+            if (gi < gpb) {
+              sz_s[gi] = sp[gi];
+              sz_z[gi] = zp[gi];
+            }
           }
         }
         tc_fence_after();
-        const int total = nb * gpb;  // group accumulators of the batch
-        for (int i0 = 0; i0 < total; i0 += kLoads) {
+        const int kvalid = min(kBK, a.K - (kb0 + j) * kBK);
+        // the group accumulators of the block are read in batches of GB groups
+        // with one wait per batch (each wait is a round trip to tensor memory)
+        constexpr int LD = MV <= 8 ? 8 : MV;  // columns loaded per group
+        constexpr int GB = 4 * LD <= 32 ? 4 : (2 * LD <= 32 ? 2 : 1);
 #pragma unroll
-          for (int t = 0; t < kLoads; ++t) {
-            const int i = i0 + t;
-            if (i < total) {
-              const int b = i / gpb, gi = i - b * gpb;
-              const int j = j0 + 4 * b;
-              if (gi * g < min(kBK, a.K - (kb0 + j) * kBK)) {
-                tmem_ld_32x32b<LD>(tmem + trow + kDCol + ((j & (ndb - 1)) * gpb + gi) * MPAD, dv[t]);
-                if (a.sz_tma) {
-                  const int zs = (j / spb) % kSzSlots;
-                  const uint16_t* sp =
-                      reinterpret_cast<const uint16_t*>(szring + zs * L::kSzSlotBytes) + r * 8 + (j % spb) * gpb + gi;
-                  scv[t] = __uint_as_float(uint32_t(sp[0]) << 16);
-                  zcv[t] = __uint_as_float(uint32_t(sp[L::kSzSlotBytes / 4]) << 16);
-                } else {
-                  scv[t] = __uint_as_float(sz_s[gi] << 16);
-                  zcv[t] = __uint_as_float(sz_z[gi] << 16);
-                }
-                ++n;
-              }
-            }
-          }
-          tmem_ld_wait();
+        for (int gi0 = 0; gi0 < 4; gi0 += GB) {
+          if (gi0 < gpb) {
+            uint32_t dv[GB][LD];
 #pragma unroll
-          for (int t = 0; t < kLoads; ++t) {
-            const int i = i0 + t;
-            if (i < total) {
-              const int b = i / gpb, gi = i - b * gpb;
-              const int j = j0 + 4 * b;
-              if (gi * g < min(kBK, a.K - (kb0 + j) * kBK)) {
+            for (int b = 0; b < GB; ++b)
+              if (gi0 + b < gpb && (gi0 + b) * g < kvalid)
+                tmem_ld_32x32b<LD>(tmem + trow + kDCol + (db * gpb + gi0 + b) * MPAD, dv[b]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int b = 0; b < GB; ++b) {
+              const int gi = gi0 + b;
+              if (gi < gpb && gi * g < kvalid) {
+                const float sc = __uint_as_float(sz_s[gi] << 16);
+                const float zc = __uint_as_float(sz_z[gi] << 16);
                 const float* xg = xs + ((j % kXsSlots) * 4 + gi) * MV;
                 // accumulators hold sum((128 + q) x): s * D + (z - 128 s) * X
-                const float zc2 = fmaf(-128.f, scv[t], zcv[t]);
+                const float zc2 = fmaf(-128.f, sc, zc);
 #pragma unroll
-                for (int m = 0; m < MV; ++m) acc[m] = fmaf(scv[t], __uint_as_float(dv[t][m]), fmaf(zc2, xg[m], acc[m]));
+                for (int m = 0; m < MV; ++m) acc[m] = fmaf(sc, __uint_as_float(dv[b][m]), fmaf(zc2, xg[m], acc[m]));
               }
             }
           }
         }
-        (void)n;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          for (int b = 0; b < nb; ++b) {
-            const int j = j0 + 4 * b;
-            mbar_arrive(&dempty[j & (ndb - 1)]);
-            if (a.sz_tma) mbar_arrive(&szfree[(j / spb) % kSzSlots]);
-          }
+          mbar_arrive(&dempty[db]);
+          if (a.sz_tma) mbar_arrive(&szfree[zs]);
         }
       }
       return true;
     };
-    // blocks folded per batch: what the accumulator ring allows (the MMAs of
-    // block j wait for the fold of block j - ndb, so 4 * batch <= ndb), and
-    // few enough that the batch's first block is folded before its stage's
-    // mdone barrier can complete again: that needs the folding warps' own
-    // dequantization of block j0 + NW, so 4 * (batch - 1) + lag < NW suffices.
-    // Scales and zeros of earlier blocks come from the staged boxes only.
-    const int fold_batch =
-        (kInt4 && a.sz_tma) ? max(1, min(min(ndb / 4, max(1, kLoads / gpb)), (NW - 1 - lag) / 4 + 1)) : 1;
-    int next_fold = u;  // first block of this warp group not yet folded
     if constexpr (kTmemA) {
       for (int j = 0; j < nkb && !failed; ++j) {
         const int s = j % NW;
@@ -506,21 +480,13 @@ __global__ void __launch_bounds__(kThreads, 1) wq_gemm_kernel(const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(&xready[j % kXsSlots]);
           }
-          // fold a batch of this group's blocks once its last block is `lag` behind
           const int jf = j - lag;
-          if (jf >= 0 && (jf & 3) == u && ((jf - u) / 4) % fold_batch == fold_batch - 1) {
-            if (!fold_blocks(next_fold, (jf - next_fold) / 4 + 1)) { failed = true; break; }
-            next_fold = jf + 4;
-          }
+          if (jf >= 0 && (jf & 3) == u && !fold_block(jf)) { failed = true; break; }
         }
       }
       if constexpr (kInt4) {
-        // the blocks still unfolded, in batches
-        while (!failed && next_fold < nkb) {
-          const int nb = min(fold_batch, (nkb - 1 - next_fold) / 4 + 1);
-          if (!fold_blocks(next_fold, nb)) failed = true;
-          next_fold += 4 * nb;
-        }
+        for (int jf = max(0, nkb - lag); jf < nkb && !failed; ++jf)
+          if ((jf & 3) == u && !fold_block(jf)) failed = true;
       }
     }
     if constexpr (!kInt4) {

@@ -452,18 +452,13 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
         load_x_smem<FMT, MM>(xr, st + kRB * F::kRowBytes, lane, p.c * kChunkK + lane * F::kLaneK < a.K);
         cur_c = p.c;
       }
-      // all J rows of this warp at once: independent chains interleave.  Rows
-      // past the stage's last row are skipped (the test is uniform across the
-      // warp); their partials are zero and never stored.
+      // all J rows of this warp at once: independent chains interleave.  A full
+      // stage runs every row without a test; in a partial stage (the last rows
+      // of a CTA) rows past its end are skipped, the test uniform across the
+      // warp, and their partials are zero and never stored.
       float acc[J][MM];
-#pragma unroll
-      for (int j = 0; j < J; ++j) {
+      auto row_dot = [&](int j) {
         const int i = cw + j * CWN;
-        if (i >= rows) {
-#pragma unroll
-          for (int m = 0; m < MM; ++m) acc[j][m] = 0.f;
-          continue;
-        }
         if constexpr (FMT == WQ_FP6_E3M2)
           lane_dot<FMT, MM>(st + i * 512, st + kRB * 512 + i * 256, lane, xr, dc, acc[j]);
         else
@@ -474,6 +469,20 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
           const float zc = __uint_as_float(zz[j] << 16);
 #pragma unroll
           for (int m = 0; m < MM; ++m) acc[j][m] = fmaf(sc, acc[j][m], zc * xr.xsum[m]);
+        }
+      };
+      if (rows == kRB) {
+#pragma unroll
+        for (int j = 0; j < J; ++j) row_dot(j);
+      } else {
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+          if (cw + j * CWN < rows) {
+            row_dot(j);
+          } else {
+#pragma unroll
+            for (int m = 0; m < MM; ++m) acc[j][m] = 0.f;
+          }
         }
       }
       // every lane's shared-memory reads of the stage are done: release them on
