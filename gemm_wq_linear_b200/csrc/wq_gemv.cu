@@ -13,16 +13,22 @@
 //    fixed order: the result is deterministic).
 //  * K is cut into chunks of 32 lanes x LANE_K weights.  A stage of the
 //    shared-memory ring holds one chunk of kJ rows per consumer warp plus, for
-//    a chunk's first stage, that chunk of x.  A producer warp (or, without one,
-//    the last consumer warp out of the stage) fills the ring with 2-D tensor
-//    copies of 8-row boxes and bulk copies of x, completing on the stage's
-//    mbarrier, far ahead of the consumers.
+//    a chunk's first stage, that chunk of x, and (int4, when a row of scales is
+//    a multiple of 16 bytes) the scales and zeros of the stage's rows.  A
+//    producer warp (or, without one, the last consumer warp out of the stage)
+//    fills the ring with 2-D tensor copies of 8-row boxes and bulk copies of x,
+//    completing on the stage's mbarrier, ahead of the consumers.
+//  * With a producer, a converter warp takes the stages in order as they land,
+//    converts each chunk of x once per CTA, in place, to the packed fp32 pairs
+//    the consumer lanes multiply with (int4: pre-scaled, plus each lane's sum),
+//    and releases the stage on a second mbarrier; the consumers copy them into
+//    registers, where they stay for the whole chunk.  Without a producer
+//    (M >= 3) every consumer warp converts x itself.
 //  * Each consumer lane reads its 16 bytes (FP6: 16 + 8) of a row from shared
 //    memory, decodes them in registers (explicit LOP3 / funnel-shift / PRMT PTX,
-//    decode.cuh) and multiplies with its activations, held in registers for the
-//    whole chunk, with the packed fp32 FMA.  Lane partials accumulate in shared
-//    memory across stages (M <= 2) or are reduced with shuffles per stage
-//    (M >= 3); the sums are scaled and rounded to bf16 once.
+//    decode.cuh) and multiplies with the packed fp32 FMA.  Lane partials
+//    accumulate in shared memory across stages (M <= 2) or are reduced with
+//    shuffles per stage (M >= 3); the sums are scaled and rounded to bf16 once.
 //
 // Dequantization arithmetic (fp32 accumulation):
 //  * int4: decoded value q * 2^(p - 8) against activations scaled by 2^(8 - p)
@@ -67,13 +73,13 @@ struct GemvFmt<WQ_BF16> {
 
 constexpr int kJ = 4;  // rows of a stage each consumer warp takes
 // Launch shape per format and M (measured on B200):
-//  * M = 1, int4 / int8 / bf16: two CTAs per SM, each with eight consumer warps
-//    and a producer warp that keeps the ring full; the next layer's CTAs can
-//    start while the last CTAs of this one drain (programmatic dependent launch);
-//  * M = 1, FP6 (decode-bound): one CTA per SM with sixteen consumer warps and a
-//    producer, so every SM carries the same share;
-//  * M = 2: one CTA per SM, eight consumer warps and a producer (168 registers a
-//    thread);
+//  * M = 1, int4 / int8 / bf16: two CTAs per SM, each with eight consumer warps,
+//    a producer warp that keeps the ring full and a converter warp; the next
+//    layer's CTAs can start while the last CTAs of this one drain (programmatic
+//    dependent launch);
+//  * M = 1, FP6 (decode-bound): one CTA per SM with sixteen consumer warps, a
+//    producer and a converter, so every SM carries the same share;
+//  * M = 2: one CTA per SM, eight consumer warps, a producer and a converter;
 //  * M >= 3: one CTA per SM, eight consumer warps and no producer, so each thread
 //    may hold up to 255 registers (the activations of a chunk need them); the
 //    last warp to finish a stage refills its slot.
@@ -82,17 +88,36 @@ __host__ __device__ constexpr bool gemv_has_producer(int, int mm) { return mm <=
 __host__ __device__ constexpr int gemv_cw(int fmt, int mm) { return (mm == 1 && fmt == WQ_FP6_E3M2) ? 16 : 8; }
 __host__ __device__ constexpr int gemv_rb(int fmt, int mm) { return kJ * gemv_cw(fmt, mm); }
 __host__ __device__ constexpr int gemv_ctas_per_sm(int fmt, int mm) { return (mm == 1 && fmt != WQ_FP6_E3M2) ? 2 : 1; }
+// warps: producer and converter (when there is a producer), then the consumers
 __host__ __device__ constexpr int gemv_threads(int fmt, int mm) {
-  return 32 * (gemv_cw(fmt, mm) + (gemv_has_producer(fmt, mm) ? 1 : 0));
+  return 32 * (gemv_cw(fmt, mm) + (gemv_has_producer(fmt, mm) ? 2 : 0));
 }
 __host__ __device__ constexpr bool gemv_lane_partials(int mm) { return mm <= 2; }
 
+// One ring slot: the weights of a stage's kRB rows, then per activation row
+// the chunk's activations, then (int4 with staged scales) the scales and zeros
+// of the stage's rows.  The activation area holds the lane registers' values
+// in the order the consumers load them (pairs of packed fp32 pairs, lane after
+// lane, so that a warp's 16-byte loads are conflict-free), then the lane sums;
+// the raw bf16 chunk lands in the tail of the same area and the producer
+// converts it in place.
 template <int FMT, int MM>
 struct GemvLayout {
-  static constexpr int kChunkK = 32 * GemvFmt<FMT>::kLaneK;
-  static constexpr int kXBytes = kChunkK * 2;  // one chunk of one activation row
+  static constexpr int kLaneK = GemvFmt<FMT>::kLaneK;
+  static constexpr int kChunkK = 32 * kLaneK;
+  static constexpr int kXBytes = kChunkK * 2;   // one chunk of one activation row, bf16
   static constexpr int kRB = gemv_rb(FMT, MM);  // rows per stage
-  static constexpr int kStageBytes = (kRB * GemvFmt<FMT>::kRowBytes + MM * kXBytes + 127) / 128 * 128;
+  static constexpr int kWBytes = kRB * GemvFmt<FMT>::kRowBytes;
+  static constexpr int kPairs = kLaneK / 2;     // packed fp32 pairs per lane and activation row
+  static constexpr int kCxBytes = 32 * kPairs * 8 + 32 * 4;
+  static constexpr int kRawOff = kCxBytes - kXBytes;
+  static constexpr int kXOff = kWBytes;
+  static constexpr int kSzOff = (kXOff + MM * kCxBytes + 127) / 128 * 128;
+  static_assert(kRawOff % 16 == 0 && kCxBytes % 16 == 0 && kXOff % 128 == 0, "bulk copies need 16-byte offsets");
+  // scales then zeros of the stage's rows, gpc groups each (int4)
+  static constexpr int stage_bytes(int gpc, bool sz) {
+    return (kSzOff + (sz ? 2 * kRB * gpc * 2 : 0) + 127) / 128 * 128;
+  }
 };
 
 __device__ __forceinline__ float fp16_bits_to_float(uint16_t b) { return __half2float(__ushort_as_half(b)); }
@@ -124,13 +149,14 @@ __host__ __device__ constexpr float pow2f(int e) {
 
 // Lanes past the end of K (last chunk) get zeros: their weights are the tensor
 // copy's zero fill, so every product is zero without a per-lane branch.
+// `xs` is the raw chunk of activation row 0; row m is m * L::kCxBytes further.
 template <int FMT, int MM>
 __device__ __forceinline__ void load_x_smem(XRegs<FMT, MM>& xr, const uint8_t* xs, int lane, bool valid) {
   using L = GemvLayout<FMT, MM>;
   constexpr int LK = GemvFmt<FMT>::kLaneK;
 #pragma unroll
   for (int m = 0; m < MM; ++m) {
-    const uint8_t* base = xs + m * L::kXBytes + lane * LK * 2;
+    const uint8_t* base = xs + m * L::kCxBytes + lane * LK * 2;
     float xf[LK];
 #pragma unroll
     for (int q = 0; q < LK / 8; ++q) {
@@ -169,6 +195,45 @@ __device__ __forceinline__ void load_x_smem(XRegs<FMT, MM>& xr, const uint8_t* x
   }
 }
 
+// Producer warp: converts the raw chunk at the tail of the activation area
+// `cx` into the lane-register layout, in place (every lane has read its raw
+// values before any lane writes).  The fence orders these generic writes before
+// the tensor copies that later refill the slot.
+template <int FMT, int MM>
+__device__ __forceinline__ void convert_x(uint8_t* cx, int lane, bool valid) {
+  using L = GemvLayout<FMT, MM>;
+  XRegs<FMT, MM> xr;
+  load_x_smem<FMT, MM>(xr, cx + L::kRawOff, lane, valid);
+  __syncwarp();
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    uint8_t* row = cx + m * L::kCxBytes;
+#pragma unroll
+    for (int q = 0; q < L::kPairs / 2; ++q)
+      *reinterpret_cast<ulonglong2*>(row + (q * 32 + lane) * 16) =
+          make_ulonglong2(xr.v2[m][2 * q], xr.v2[m][2 * q + 1]);
+    if constexpr (FMT == WQ_INT4) *reinterpret_cast<float*>(row + L::kPairs * 256 + lane * 4) = xr.xsum[m];
+  }
+  fence_proxy_async_shared();
+}
+
+// Consumer: the lane's activation registers of a chunk converted by the producer.
+template <int FMT, int MM>
+__device__ __forceinline__ void load_cx(XRegs<FMT, MM>& xr, const uint8_t* cx, int lane) {
+  using L = GemvLayout<FMT, MM>;
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    const uint8_t* row = cx + m * L::kCxBytes;
+#pragma unroll
+    for (int q = 0; q < L::kPairs / 2; ++q) {
+      const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(row + (q * 32 + lane) * 16);
+      xr.v2[m][2 * q] = v.x;
+      xr.v2[m][2 * q + 1] = v.y;
+    }
+    if constexpr (FMT == WQ_INT4) xr.xsum[m] = *reinterpret_cast<const float*>(row + L::kPairs * 256 + lane * 4);
+  }
+}
+
 template <int FMT>
 struct DecodeConsts {
   Int4PairConsts i4;
@@ -176,7 +241,7 @@ struct DecodeConsts {
 };
 template <int FMT>
 __device__ __forceinline__ DecodeConsts<FMT> make_decode_consts() {
-  DecodeConsts<FMT> d;
+  DecodeConsts<FMT> d{};
   if constexpr (FMT == WQ_INT4) d.i4 = int4_pair_consts();
   if constexpr (FMT == WQ_INT8) d.i8 = int8_f32_bias();
   return d;
@@ -277,7 +342,10 @@ __device__ __forceinline__ void advance(StagePos& p, int NS, int NRB, int clo, i
   }
 }
 
-template <int FMT, int MM>
+// SZ (int4 only): the scales and zeros of each stage's rows travel with its
+// weights by tensor copies; otherwise each consumer lane loads its own one
+// stage ahead.
+template <int FMT, int MM, bool SZ>
 __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, MM)) gemv_kernel(const __grid_constant__ GemvParams a) {
   using F = GemvFmt<FMT>;
   using L = GemvLayout<FMT, MM>;
@@ -287,11 +355,14 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
   constexpr int kRB = L::kRB;
   extern __shared__ __align__(1024) uint8_t smem[];
 
+  static_assert(!SZ || FMT == WQ_INT4, "staged scales are an int4 layout");
   const int NS = a.stages;
+  const int SB = a.stage_bytes;
   uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(NS) * L::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(NS) * SB);
   uint64_t* empty = full + NS;                          // [NS] warps finished reading the slot's stage
-  int* done_cnt = reinterpret_cast<int*>(empty + NS);  // [NS] arrivals counted, to elect the refilling warp
+  uint64_t* xready = empty + NS;                        // [NS] producer: the stage was handed over (x converted)
+  int* done_cnt = reinterpret_cast<int*>(xready + NS);  // [NS] arrivals counted, to elect the refilling warp
   int* last_issued = done_cnt + NS;                    // [NS] stage last issued into the slot
   // partial sums.  Lane partials (M <= 2): [R][MM][32 lanes], each (row, lane)
   // entry owned by one thread, so stages add into it with no cross-lane step and
@@ -316,6 +387,9 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t policy = l2_policy_evict_first();
+  // int4: log2 of the group size, groups per chunk
+  const int gshift = (FMT == WQ_INT4) ? __ffs(a.groupsize) - 1 : 0;
+  const int gpc = kChunkK >> gshift;
 
   // Issue the tensor copies of one stage into its slot (one thread).  The x of a
   // chunk travels with the chunk's first stage only.
@@ -323,9 +397,10 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
     const int rows = min(kRB, R - p.rb * kRB);
     const int nbox = (rows + a.box_rows - 1) / a.box_rows;
     const int kc = min(kChunkK, a.K - p.c * kChunkK);
-    mbar_arrive_expect_tx(&full[p.slot],
-                          uint32_t(nbox * a.box_rows * F::kRowBytes) + (p.rb == 0 ? MM * uint32_t(kc) * 2 : 0u));
-    uint8_t* st = ring + size_t(p.slot) * L::kStageBytes;
+    uint32_t bytes = uint32_t(nbox * a.box_rows * F::kRowBytes) + (p.rb == 0 ? MM * uint32_t(kc) * 2 : 0u);
+    if constexpr (SZ) bytes += uint32_t(nbox * a.box_rows * gpc * 4);
+    mbar_arrive_expect_tx(&full[p.slot], bytes);
+    uint8_t* st = ring + size_t(p.slot) * SB;
     const int row0 = n0 + p.rb * kRB;
     for (int b = 0; b < nbox; ++b) {
       const int row = row0 + b * a.box_rows;
@@ -335,13 +410,18 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
       } else {
         tma_load_2d(st + b * a.box_rows * F::kRowBytes, &a.tm_w, p.c * (F::kRowBytes / 4), row, &full[p.slot], policy);
       }
+      if constexpr (SZ) {
+        uint8_t* sz = st + L::kSzOff + b * a.box_rows * gpc * 2;
+        tma_load_2d(sz, &a.tm_s, p.c * gpc, row, &full[p.slot], policy);
+        tma_load_2d(sz + kRB * gpc * 2, &a.tm_z, p.c * gpc, row, &full[p.slot], policy);
+      }
     }
   };
   auto issue_x = [&](const StagePos& p) {
     if (p.rb != 0) return;
     const int kc = min(kChunkK, a.K - p.c * kChunkK);
     for (int m = 0; m < MM; ++m)
-      bulk_g2s(ring + size_t(p.slot) * L::kStageBytes + kRB * F::kRowBytes + m * L::kXBytes,
+      bulk_g2s(ring + size_t(p.slot) * SB + L::kXOff + m * L::kCxBytes + L::kRawOff,
                a.x + size_t(m) * a.K + size_t(p.c) * kChunkK, uint32_t(kc) * 2, &full[p.slot]);
   };
 
@@ -353,12 +433,17 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], CWN);
+      mbar_init(&xready[s], 32);
       done_cnt[s] = 0;
       last_issued[s] = -1;
     }
     fence_mbar_init();
     prefetch_tmap(&a.tm_w);
     if (FMT == WQ_FP6_E3M2) prefetch_tmap(&a.tm_w2);
+    if (SZ) {
+      prefetch_tmap(&a.tm_s);
+      prefetch_tmap(&a.tm_z);
+    }
     if constexpr (!kProducer) {
       // first ring fill: weights at once; x after the previous kernel (which may
       // write it) has finished, under programmatic dependent launch
@@ -380,7 +465,7 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
 
   bool failed = false;
   if (kProducer && warp == 0) {
-    // ------------------------------------------------------------ producer (M = 1)
+    // ------------------------------------------------------------ producer (M <= 2)
     if (lane == 0) {
       StagePos p = {0, 0u, 0, c_rot};
       for (int t = 0; t < T; ++t) {
@@ -406,23 +491,43 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
       if (failed && a.pdl) pdl_wait();
     }
     __syncwarp();
+  } else if (kProducer && warp == 1) {
+    // ------------------------------------------------------------ converter (M <= 2)
+    // Takes the stages in order as they land: converts the activations of a
+    // chunk's first stage and releases every stage to the consumers on its
+    // xready barrier.  Consumers wait for xready at every stage, so a slot is
+    // never refilled before the converter has passed it.
+    StagePos u = {0, 0u, 0, c_rot};
+    for (int t = 0; t < T; ++t) {
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[u.slot], u.phase))) {
+        failed = true;
+        break;
+      }
+      if (u.rb == 0)
+        convert_x<FMT, MM>(ring + size_t(u.slot) * SB + L::kXOff, lane, u.c * kChunkK + lane * F::kLaneK < a.K);
+      mbar_arrive(&xready[u.slot]);
+      advance(u, NS, NRB, CLO, CHI);
+    }
   } else {
     // ------------------------------------------------------------ consumers
-    const int cw = kProducer ? warp - 1 : warp;
+    const int cw = kProducer ? warp - 2 : warp;
     if (a.pdl) pdl_wait();
     int cur_c = -1;
     XRegs<FMT, MM> xr;
     const DecodeConsts<FMT> dc = make_decode_consts<FMT>();
     constexpr int J = kJ;
-    const int gshift = (FMT == WQ_INT4) ? __ffs(a.groupsize) - 1 : 0;
     const int G = (FMT == WQ_INT4) ? (a.K >> gshift) : 0;
-    // int4: raw 16-bit scale and zero of this warp's rows at the lane's group,
-    // fetched one stage ahead into the other of two register sets; the load
-    // zero-extends, so no instruction touches them before the fold a stage later
-    // (rows past N are skipped: only the last CTA has them)
+    // int4 without staged scales: raw 16-bit scale and zero of this warp's rows
+    // at the lane's group, fetched one stage ahead into the other of two register
+    // sets; the load zero-extends, so no instruction touches them before the fold
+    // a stage later (rows past N are skipped: only the last CTA has them)
     const int G8 = G * CWN;
+    // int4 with staged scales: the lane's group in the stage's [kRB][gpc] arrays
+    const int sz_lane = (FMT == WQ_INT4) ? (cw * gpc + ((lane * F::kLaneK) >> gshift)) * 2 : 0;
+    const int sz_row = CWN * gpc * 2;
+    const int sz_zero = kRB * gpc * 2;
     auto fetch_sz = [&](const StagePos& p, uint32_t (&ds)[J], uint32_t (&dz)[J]) {
-      if constexpr (FMT == WQ_INT4) {
+      if constexpr (FMT == WQ_INT4 && !SZ) {
         const int k0 = p.c * kChunkK + lane * F::kLaneK;
         const int row = n0 + p.rb * kRB + cw;
         const int off = row * G + (k0 >> gshift);
@@ -444,12 +549,18 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
                      const uint32_t (&zz)[J], uint32_t (&ss_next)[J], uint32_t (&zz_next)[J]) -> bool {
       StagePos nx = p;
       advance(nx, NS, NRB, CLO, CHI);
-      if (has_next) fetch_sz(nx, ss_next, zz_next);
+      if (!SZ && has_next) fetch_sz(nx, ss_next, zz_next);
       if (!mbar_wait(&full[p.slot], p.phase)) return false;
+      if (kProducer && !mbar_wait(&xready[p.slot], p.phase)) return false;
       const int rows = min(kRB, R - p.rb * kRB);
-      const uint8_t* st = ring + p.slot * L::kStageBytes;
+      const uint8_t* st = ring + p.slot * SB;
       if (p.c != cur_c) {
-        load_x_smem<FMT, MM>(xr, st + kRB * F::kRowBytes, lane, p.c * kChunkK + lane * F::kLaneK < a.K);
+        // a chunk's first stage (rb == 0) carries its activations
+        if constexpr (kProducer) {
+          load_cx<FMT, MM>(xr, st + L::kXOff, lane);
+        } else {
+          load_x_smem<FMT, MM>(xr, st + L::kXOff + L::kRawOff, lane, p.c * kChunkK + lane * F::kLaneK < a.K);
+        }
         cur_c = p.c;
       }
       // all J rows of this warp at once: independent chains interleave.  A full
@@ -465,8 +576,14 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
           lane_dot<FMT, MM>(st + i * F::kRowBytes, nullptr, lane, xr, dc, acc[j]);
         if constexpr (FMT == WQ_INT4) {
           // sum over the lane's 32 k (one group): s * sum(q x) + z * sum(x)
-          const float sc = __uint_as_float(ss[j] << 16);
-          const float zc = __uint_as_float(zz[j] << 16);
+          uint32_t sb = ss[j], zb = zz[j];
+          if constexpr (SZ) {
+            const uint8_t* szp = st + L::kSzOff + sz_lane + j * sz_row;
+            sb = *reinterpret_cast<const uint16_t*>(szp);
+            zb = *reinterpret_cast<const uint16_t*>(szp + sz_zero);
+          }
+          const float sc = __uint_as_float(sb << 16);
+          const float zc = __uint_as_float(zb << 16);
 #pragma unroll
           for (int m = 0; m < MM; ++m) acc[j][m] = fmaf(sc, acc[j][m], zc * xr.xsum[m]);
         }
@@ -635,7 +752,7 @@ constexpr size_t kGemvSmemPerSm = 220 * 1024;
 
 constexpr int kBoxRows = 8;
 
-template <int FMT, int MM>
+template <int FMT, int MM, bool SZ>
 static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int sm_count) {
   using L = GemvLayout<FMT, MM>;
   using F = GemvFmt<FMT>;
@@ -668,13 +785,17 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   p.chunks_per_split = CPS;
   p.rows_per_cta = R;
   p.box_rows = kBoxRows;
-  const size_t fixed = 8 * 24 + 16 + size_t(R) * part_row;
-  if (fixed + 2 * size_t(L::kStageBytes) > 200 * 1024) return cudaErrorInvalidValue;
-  int stages = fixed < kGemvSmemBudget ? int((kGemvSmemBudget - fixed) / L::kStageBytes) : 2;
+  const int gpc = FMT == WQ_INT4 ? L::kChunkK / p.groupsize : 0;
+  p.sz_tma = SZ ? 1 : 0;
+  p.stage_bytes = L::stage_bytes(gpc, SZ);
+  // barriers and counters: full, empty, xready (8 bytes each), done_cnt, last_issued (4 each) per slot
+  const size_t fixed = 8 * 32 + 16 + size_t(R) * part_row;
+  if (fixed + 2 * size_t(p.stage_bytes) > 200 * 1024) return cudaErrorInvalidValue;
+  int stages = fixed < kGemvSmemBudget ? int((kGemvSmemBudget - fixed) / p.stage_bytes) : 2;
   if (stages > 8) stages = 8;
   if (stages < 2) stages = 2;
   p.stages = stages;
-  const size_t smem = size_t(stages) * L::kStageBytes + size_t(stages) * 24 + 16 + size_t(R) * part_row;
+  const size_t smem = size_t(stages) * p.stage_bytes + size_t(stages) * 32 + 16 + size_t(R) * part_row;
 
   // tensor maps: rows of packed bytes viewed as 32-bit elements, one chunk per box
   cudaError_t e;
@@ -689,11 +810,20 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
     e = make_tmap_u32_2d(&p.tm_w, p.packed, rowb / 4, uint64_t(p.N), rowb, F::kRowBytes / 4, kBoxRows);
   }
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gemv_kernel<FMT, MM>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if constexpr (SZ) {
+    // scales / zeros [N, G] bf16: boxes of one chunk's gpc groups x 8 rows (the
+    // row pitch 2 G is a multiple of 16 bytes, checked by the caller)
+    const uint64_t G = uint64_t(p.K / p.groupsize);
+    e = make_tmap_2d(&p.tm_s, p.scales, 2, G, uint64_t(p.N), G * 2, uint32_t(gpc), kBoxRows, 0);
+    if (e == cudaSuccess) e = make_tmap_2d(&p.tm_z, p.zeros, 2, G, uint64_t(p.N), G * 2, uint32_t(gpc), kBoxRows, 0);
+    if (e != cudaSuccess) return e;
+  }
+  auto kernel = gemv_kernel<FMT, MM, SZ>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int grid = (p.N + R - 1) / R * S;
   if (S > 1) {
-    e = cudaFuncSetAttribute(gemv_kernel<FMT, MM>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
@@ -717,16 +847,26 @@ static cudaError_t launch_gemv_t(const GemvParams& p0, cudaStream_t stream, int 
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<FMT, MM>, p);
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+// int4 stages its scales and zeros by tensor copies when a row of them (K / g
+// bf16) is a multiple of 16 bytes (the arrays are 16-byte aligned by contract)
+template <int FMT, int MM>
+static cudaError_t launch_gemv_sz(const GemvParams& p, cudaStream_t s, int sm_count) {
+  if constexpr (FMT == WQ_INT4) {
+    if ((p.K / p.groupsize) % 8 == 0) return launch_gemv_t<FMT, MM, true>(p, s, sm_count);
+  }
+  return launch_gemv_t<FMT, MM, false>(p, s, sm_count);
 }
 
 template <int FMT>
 static cudaError_t launch_gemv_fmt(const GemvParams& p, cudaStream_t s, int sm_count) {
   switch (p.M) {
-    case 1: return launch_gemv_t<FMT, 1>(p, s, sm_count);
-    case 2: return launch_gemv_t<FMT, 2>(p, s, sm_count);
-    case 3: return launch_gemv_t<FMT, 3>(p, s, sm_count);
-    default: return launch_gemv_t<FMT, 4>(p, s, sm_count);
+    case 1: return launch_gemv_sz<FMT, 1>(p, s, sm_count);
+    case 2: return launch_gemv_sz<FMT, 2>(p, s, sm_count);
+    case 3: return launch_gemv_sz<FMT, 3>(p, s, sm_count);
+    default: return launch_gemv_sz<FMT, 4>(p, s, sm_count);
   }
 }
 

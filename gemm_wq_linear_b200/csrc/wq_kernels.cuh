@@ -43,6 +43,8 @@ cudaError_t gemm_take_status(uint32_t* status);
 struct GemvParams {
   CUtensorMap tm_w;        // packed weights (FP6: the 4-bit plane)
   CUtensorMap tm_w2;       // FP6: the 2-bit plane
+  CUtensorMap tm_s;        // int4 with sz_tma: scales [N, K/g] bf16, boxes of one chunk's groups x 8 rows
+  CUtensorMap tm_z;        // int4 with sz_tma: zeros, same boxes
   const uint16_t* x;       // bf16 [M, K]
   const void* packed;      // packed weights of `fmt`
   const uint16_t* scales;  // fp16 [N] (int8, FP6) or bf16 [N, K/g] (int4)
@@ -54,6 +56,8 @@ struct GemvParams {
   int chunks_per_split;    // K-chunks per split, set by the launcher
   int stages;              // shared-memory ring depth, set by the launcher
   int box_rows;            // rows per tensor-copy box (rows_per_cta is a multiple)
+  int stage_bytes;         // bytes of one ring slot, set by the launcher
+  int sz_tma;              // int4: scales / zeros staged with the weights by tensor copies
   int pdl;                 // programmatic dependent launch enabled
 };
 
