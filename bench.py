@@ -147,7 +147,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ measured DRAM traffic
 KERNEL_SOURCES = ("gemm_wq_linear_b200/csrc/wq_gemv.cu", "gemm_wq_linear_b200/csrc/decode.cuh",
-                  "gemm_wq_linear_b200/csrc/ptx.cuh")
+                  "gemm_wq_linear_b200/csrc/ptx.cuh", "gemm_wq_linear_b200/csrc/wq_kernels.cuh")
 
 
 def kernel_source_hash():

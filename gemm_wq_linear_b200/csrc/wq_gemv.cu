@@ -85,12 +85,19 @@ constexpr int kJ = 4;  // rows of a stage each consumer warp takes
 //    last warp to finish a stage refills its slot.
 // A stage holds kJ rows per consumer warp.
 __host__ __device__ constexpr bool gemv_has_producer(int, int mm) { return mm <= 2; }
+// int4 with a producer: a converter warp prepares x once per CTA (its per-lane
+// conversion, with the pre-scaling and the lane sums, is the costliest); the
+// other formats convert their few values per lane in the consumers (measured
+// 1-2 % faster than with a converter)
+__host__ __device__ constexpr bool gemv_has_converter(int fmt, int mm) {
+  return gemv_has_producer(fmt, mm) && fmt == WQ_INT4;
+}
 __host__ __device__ constexpr int gemv_cw(int fmt, int mm) { return (mm == 1 && fmt == WQ_FP6_E3M2) ? 16 : 8; }
 __host__ __device__ constexpr int gemv_rb(int fmt, int mm) { return kJ * gemv_cw(fmt, mm); }
 __host__ __device__ constexpr int gemv_ctas_per_sm(int fmt, int mm) { return (mm == 1 && fmt != WQ_FP6_E3M2) ? 2 : 1; }
-// warps: producer and converter (when there is a producer), then the consumers
+// warps: the producer, the converter, then the consumers
 __host__ __device__ constexpr int gemv_threads(int fmt, int mm) {
-  return 32 * (gemv_cw(fmt, mm) + (gemv_has_producer(fmt, mm) ? 2 : 0));
+  return 32 * (gemv_cw(fmt, mm) + (gemv_has_producer(fmt, mm) ? 1 : 0) + (gemv_has_converter(fmt, mm) ? 1 : 0));
 }
 __host__ __device__ constexpr bool gemv_lane_partials(int mm) { return mm <= 2; }
 
@@ -109,7 +116,7 @@ struct GemvLayout {
   static constexpr int kRB = gemv_rb(FMT, MM);  // rows per stage
   static constexpr int kWBytes = kRB * GemvFmt<FMT>::kRowBytes;
   static constexpr int kPairs = kLaneK / 2;     // packed fp32 pairs per lane and activation row
-  static constexpr int kCxBytes = 32 * kPairs * 8 + 32 * 4;
+  static constexpr int kCxBytes = gemv_has_converter(FMT, MM) ? 32 * kPairs * 8 + 32 * 4 : kXBytes;
   static constexpr int kRawOff = kCxBytes - kXBytes;
   static constexpr int kXOff = kWBytes;
   static constexpr int kSzOff = (kXOff + MM * kCxBytes + 127) / 128 * 128;
@@ -351,6 +358,7 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
   using L = GemvLayout<FMT, MM>;
   constexpr int kChunkK = L::kChunkK;
   constexpr bool kProducer = gemv_has_producer(FMT, MM);
+  constexpr bool kConv = gemv_has_converter(FMT, MM);
   constexpr int CWN = gemv_cw(FMT, MM);
   constexpr int kRB = L::kRB;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -491,26 +499,28 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
       if (failed && a.pdl) pdl_wait();
     }
     __syncwarp();
-  } else if (kProducer && warp == 1) {
-    // ------------------------------------------------------------ converter (M <= 2)
+  } else if (kConv && warp == 1) {
+    // ------------------------------------------------------------ converter (int4, M <= 2)
     // Takes the stages in order as they land: converts the activations of a
     // chunk's first stage and releases every stage to the consumers on its
     // xready barrier.  Consumers wait for xready at every stage, so a slot is
     // never refilled before the converter has passed it.
-    StagePos u = {0, 0u, 0, c_rot};
-    for (int t = 0; t < T; ++t) {
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[u.slot], u.phase))) {
-        failed = true;
-        break;
+    if constexpr (kConv) {
+      StagePos u = {0, 0u, 0, c_rot};
+      for (int t = 0; t < T; ++t) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[u.slot], u.phase))) {
+          failed = true;
+          break;
+        }
+        if (u.rb == 0)
+          convert_x<FMT, MM>(ring + size_t(u.slot) * SB + L::kXOff, lane, u.c * kChunkK + lane * F::kLaneK < a.K);
+        mbar_arrive(&xready[u.slot]);
+        advance(u, NS, NRB, CLO, CHI);
       }
-      if (u.rb == 0)
-        convert_x<FMT, MM>(ring + size_t(u.slot) * SB + L::kXOff, lane, u.c * kChunkK + lane * F::kLaneK < a.K);
-      mbar_arrive(&xready[u.slot]);
-      advance(u, NS, NRB, CLO, CHI);
     }
   } else {
     // ------------------------------------------------------------ consumers
-    const int cw = kProducer ? warp - 2 : warp;
+    const int cw = warp - (kProducer ? 1 : 0) - (kConv ? 1 : 0);
     if (a.pdl) pdl_wait();
     int cur_c = -1;
     XRegs<FMT, MM> xr;
@@ -551,12 +561,12 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
       advance(nx, NS, NRB, CLO, CHI);
       if (!SZ && has_next) fetch_sz(nx, ss_next, zz_next);
       if (!mbar_wait(&full[p.slot], p.phase)) return false;
-      if (kProducer && !mbar_wait(&xready[p.slot], p.phase)) return false;
+      if (kConv && !mbar_wait(&xready[p.slot], p.phase)) return false;
       const int rows = min(kRB, R - p.rb * kRB);
       const uint8_t* st = ring + p.slot * SB;
       if (p.c != cur_c) {
         // a chunk's first stage (rb == 0) carries its activations
-        if constexpr (kProducer) {
+        if constexpr (kConv) {
           load_cx<FMT, MM>(xr, st + L::kXOff, lane);
         } else {
           load_x_smem<FMT, MM>(xr, st + L::kXOff + L::kRawOff, lane, p.c * kChunkK + lane * F::kLaneK < a.K);
@@ -693,50 +703,8 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
       }
     }
   }
-  if constexpr (kLanePart) {
-    if (S > 1) {
-      // every CTA of the cluster reaches both cluster barriers, failed or not
-      cluster_sync_all();  // all lane partials of the cluster are final
-      if (rank == 0 && !any_failed) {
-        for (int idx = threadIdx.x; idx < R * MM; idx += blockDim.x) {
-          const int r = idx / MM;
-          const int m = idx - r * MM;
-          const uint32_t base = smem_u32(part + idx * 32);
-          float v = 0.f;
-          for (int q = 0; q < S; ++q) {
-            const uint32_t src = q == 0 ? base : map_to_rank(base, uint32_t(q));
-            for (int l = 0; l < 32; ++l) v += ld_cluster_f32(src + 4 * ((l + idx) & 31));
-          }
-          const int n = n0 + r;
-          if constexpr (FMT == WQ_INT8) {
-            v *= fp16_bits_to_float(a.scales[n]);
-          } else if constexpr (FMT == WQ_FP6_E3M2) {
-            v = (v * 0x1p124f) * fp16_bits_to_float(a.scales[n]);
-          }
-          a.y[size_t(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-        }
-      }
-      cluster_sync_all();  // keep every CTA's shared memory until rank 0 has read it
-      return;
-    }
-  }
-  if (any_failed) return;
-  // sum the partials of each (row, activation row) in a fixed order: the 32 lane
-  // partials (starting at a rotating lane so that neighbouring threads read
-  // different banks), or the per-chunk values in chunk order
-  for (int idx = threadIdx.x; idx < R * MM; idx += blockDim.x) {
-    int r, m;
-    float v = 0.f;
-    if constexpr (kLanePart) {
-      r = idx / MM;
-      m = idx - r * MM;
-      const float* src = part + idx * 32;
-      for (int l = 0; l < 32; ++l) v += src[(l + idx) & 31];
-    } else {
-      m = idx / R;
-      r = idx - m * R;
-      for (int c = 0; c < C; ++c) v += part[(c * R + r) * MM + m];
-    }
+  // scale of a finished sum, rounding to bf16 and the store
+  auto store_y = [&](int r, int m, float v) {
     const int n = n0 + r;
     if constexpr (FMT == WQ_INT8) {
       v *= fp16_bits_to_float(a.scales[n]);
@@ -744,6 +712,64 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
       v = (v * 0x1p124f) * fp16_bits_to_float(a.scales[n]);
     }
     a.y[size_t(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  };
+  // sum of a warp's 32 lane values by a fixed shuffle tree (every lane ends with
+  // the same, deterministic total)
+  auto warp_sum = [](float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+  };
+  const int nwarps = int(blockDim.x) >> 5;
+  if constexpr (kLanePart) {
+    if (S > 1) {
+      // every CTA of the cluster reaches both cluster barriers, failed or not
+      cluster_sync_all();  // all lane partials of the cluster are final
+      if (!any_failed) {
+        // rank q finishes its slice of the rows, one warp per (row, activation
+        // row): lane l adds the S CTAs' partials of lane l in rank order (the
+        // loads are issued together), then the shuffle tree sums the lanes
+        const int RS = (R + S - 1) / S;
+        const int lo = rank * RS * MM, hi = min(R, (rank + 1) * RS) * MM;
+        for (int idx = lo + warp; idx < hi; idx += nwarps) {
+          const uint32_t base = smem_u32(part + idx * 32 + lane);
+          float pv[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q < S) pv[q] = ld_cluster_f32(map_to_rank(base, uint32_t(q)));
+          float v = 0.f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q < S) v += pv[q];
+          v = warp_sum(v);
+          if (lane == 0) store_y(idx / MM, idx % MM, v);
+        }
+      }
+      cluster_sync_all();  // keep every CTA's shared memory until all ranks have read it
+      return;
+    }
+  }
+  if (any_failed) return;
+  if constexpr (kLanePart) {
+    // one thread per (row, activation row): its 32 lane partials in a fixed
+    // order, starting at a rotating lane so that neighbouring threads read
+    // different banks (a warp per row with a shuffle tree measured slower here:
+    // with many rows per CTA its dependent shuffles serialise)
+    for (int idx = threadIdx.x; idx < R * MM; idx += blockDim.x) {
+      const float* src = part + idx * 32;
+      float v = 0.f;
+      for (int l = 0; l < 32; ++l) v += src[(l + idx) & 31];
+      store_y(idx / MM, idx % MM, v);
+    }
+  } else {
+    // the per-chunk values in chunk order
+    for (int idx = threadIdx.x; idx < R * MM; idx += blockDim.x) {
+      const int m = idx / R;
+      const int r = idx - m * R;
+      float v = 0.f;
+      for (int c = 0; c < C; ++c) v += part[(c * R + r) * MM + m];
+      store_y(r, m, v);
+    }
   }
 }
 
