@@ -151,11 +151,15 @@ KERNEL_SOURCES = ("gemm_wq_linear_b200/csrc/wq_gemv.cu", "gemm_wq_linear_b200/cs
 
 
 def kernel_source_hash():
+    """Hash of the GEMV sources with // comments and whitespace removed, so that
+    a comment edit does not invalidate a traffic capture of the same code."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            code = re.sub(r"//[^\n]*", "", f.read())
+        h.update(re.sub(r"\s+", " ", code).encode())
     return h.hexdigest()[:16]
 
 

@@ -8,9 +8,9 @@
 // reads each packed byte exactly once and hides dequantization under the stream:
 //
 //  * A CTA owns a block of R output rows over its share of K.  When R would not
-//    fill one stage (small N), a thread-block cluster splits K and rank 0 sums
-//    the cluster's partials through distributed shared memory (no scratch, a
-//    fixed order: the result is deterministic).
+//    fill one stage (small N), a thread-block cluster splits K and its CTAs sum
+//    the cluster's partials through distributed shared memory, each finishing a
+//    slice of the rows (no scratch, a fixed order: the result is deterministic).
 //  * K is cut into chunks of 32 lanes x LANE_K weights.  A stage of the
 //    shared-memory ring holds one chunk of kJ rows per consumer warp plus, for
 //    a chunk's first stage, that chunk of x, and (int4, when a row of scales is
@@ -380,7 +380,8 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
   float* part = reinterpret_cast<float*>(last_issued + NS + (NS & 1));
   const int C = (a.K + kChunkK - 1) / kChunkK;
   // split K: the S CTAs of a cluster share a row block, rank q taking chunks
-  // [CLO, CHI); rank 0 sums the cluster's partials at the end
+  // [CLO, CHI); at the end rank q sums the cluster's partials of its slice of
+  // the rows
   const int S = a.ksplit;
   const int rank = blockIdx.x % S;
   const int n0 = (blockIdx.x / S) * a.rows_per_cta;
