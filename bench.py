@@ -159,7 +159,7 @@ def kernel_source_hash():
     for rel in KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel)) as f:
             code = re.sub(r"//[^\n]*", "", f.read())
-        h.update(re.sub(r"\s+", " ", code).encode())
+        h.update(re.sub(r"\s+", " ", code).strip().encode())
     return h.hexdigest()[:16]
 
 

@@ -1,0 +1,72 @@
+"""Host-side logic of bench.py, on CPU: the algorithmic byte count, the workload
+shapes and the source hash that ties a committed traffic capture to the code.
+"""
+
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import gemm_wq_linear_b200 as wq  # noqa: E402
+
+WORKLOADS = ["llama2-7b-int4-m1", "llama2-7b-stack-int4-g32-m1", "int8-4096-m1", "llama-70b-fp6-m1",
+             "llama-70b-fp6-m8", "opt-30b-int8-m1", "opt-30b-bf16-m1", "opt-30b-fp6-m32", "opt-30b-int4-g128-m8"]
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_algorithmic_bytes_equal_the_library_buffers(name):
+    """bench.py's byte count per call = the buffers the library sizes (packed
+    weight, scales, int4 zeros) + x + y, for every layer of every workload."""
+    for _, fmt, g, K, N, M in bench.workload_layers(name):
+        sz = wq.wq_scales_size(fmt, N, K, g)
+        lib = wq.wq_packed_size(fmt, N, K) + sz * (2 if fmt == "int4" else 1) + 2 * M * K + 2 * M * N
+        assert bench.algo_bytes(fmt, g, K, N, M) == lib
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_workload_shapes_meet_the_abi(name):
+    """Every benchmarked layer has K a multiple of 64 and N of 8 (16-byte packed
+    rows and outputs), int4 groups that divide K, and M within 1..32."""
+    layers = bench.workload_layers(name)
+    assert layers
+    for _, fmt, g, K, N, M in layers:
+        assert K % 64 == 0 and N % 8 == 0 and 1 <= M <= 32
+        if fmt == "int4":
+            assert g in (32, 64, 128) and K % g == 0
+
+
+def test_stack_is_32_layers_of_the_7b_set():
+    default = bench.workload_layers("llama2-7b-int4-m1")
+    stack = bench.workload_layers("llama2-7b-stack-int4-g32-m1")
+    assert len(default) == 8 and len(stack) == 128
+    g32 = [ly[1:] for ly in default if ly[2] == 32]
+    assert [ly[1:] for ly in stack[:4]] == g32 and [ly[1:] for ly in stack[-4:]] == g32
+
+
+def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    src = tmp_path / "k.cu"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", ("k.cu",))
+    src.write_text("int f(int a) {\n  return a + 1;  // one\n}\n")
+    h0 = bench.kernel_source_hash()
+    src.write_text("// a header comment\nint f(int a)   {\n\n  return a + 1;  // another note\n}\n")
+    assert bench.kernel_source_hash() == h0
+    src.write_text("int f(int a) {\n  return a + 2;\n}\n")
+    assert bench.kernel_source_hash() != h0
+
+
+def test_measured_traffic_needs_a_matching_hash(tmp_path, monkeypatch):
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "k.cu").write_text("int g;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", ("k.cu",))
+    prof = tmp_path / "profiles" / "gemv_w_traffic.md"
+    prof.write_text(f"traffic_bytes_per_launch: 1234\nkernel_source_hash: {bench.kernel_source_hash()}\n")
+    assert bench.measured_traffic("w") == 1234.0
+    prof.write_text("traffic_bytes_per_launch: 1234\nkernel_source_hash: 0000000000000000\n")
+    assert bench.measured_traffic("w") is None
+    assert bench.measured_traffic("missing") is None
