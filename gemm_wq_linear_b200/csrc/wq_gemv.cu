@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
   uint8_t* ring = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(NS) * SB);
   uint64_t* empty = full + NS;                          // [NS] warps finished reading the slot's stage
-  uint64_t* xready = empty + NS;                        // [NS] producer: the stage was handed over (x converted)
+  uint64_t* xready = empty + NS;                        // [NS] converter: the stage was handed over (x converted)
   int* done_cnt = reinterpret_cast<int*>(xready + NS);  // [NS] arrivals counted, to elect the refilling warp
   int* last_issued = done_cnt + NS;                    // [NS] stage last issued into the slot
   // partial sums.  Lane partials (M <= 2): [R][MM][32 lanes], each (row, lane)
@@ -400,8 +400,9 @@ __global__ void __launch_bounds__(gemv_threads(FMT, MM), gemv_ctas_per_sm(FMT, M
   const int gshift = (FMT == WQ_INT4) ? __ffs(a.groupsize) - 1 : 0;
   const int gpc = kChunkK >> gshift;
 
-  // Issue the tensor copies of one stage into its slot (one thread).  The x of a
-  // chunk travels with the chunk's first stage only.
+  // Issue the tensor copies of one stage into its slot (one thread): the weight
+  // boxes and, with SZ, the scale and zero boxes of the same rows.  The x of a
+  // chunk travels with the chunk's first stage only (issue_x).
   auto issue_w = [&](const StagePos& p) {
     const int rows = min(kRB, R - p.rb * kRB);
     const int nbox = (rows + a.box_rows - 1) / a.box_rows;
