@@ -267,6 +267,43 @@ def oracle_sample_run(layers, budget_s):
     return nbytes / dt / 1e9, cores, desc
 
 
+def cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
+def cpu_baseline(layers, budget_s):
+    """The oracle timed on the host: with every thread NumPy's BLAS uses on the
+    cores this process may run on, then with one thread (half the budget)."""
+    v, cores, desc = oracle_sample_run(layers, budget_s)
+    out = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc, "cpu_model": cpu_model(),
+           "affinity_cores": len(os.sched_getaffinity(0))}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            v1, _, desc1 = oracle_sample_run(layers, budget_s / 2)
+        out["single_thread"] = {"value": v1, "unit": "GB/s", "cores": 1, "sample": desc1}
+    except ImportError:
+        pass
+    return out
+
+
+def derived_rates(layers, ms, world):
+    """Rates derived from the device time of one step: the bf16-equivalent
+    weight rate (2 N K bytes a layer, as if the weights were unquantized bf16)."""
+    bf16_bytes = sum(2 * N * K for (_, _, _, K, N, _) in layers)
+    return {"bf16_equivalent_gbps": world * bf16_bytes / (ms * 1e-3) / 1e9,
+            "note": "2*N*K bytes per layer / device time: the rate an unquantized bf16 layer would need"}
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -478,10 +515,11 @@ def main():
                    "parallelism": f"replicas x{world}"},
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "frac": achieved / peak, "peak_kind": peak_kind, "frac_of_datasheet_8000": achieved / 8000.0,
                      "traffic": None if args.layer else measured_traffic(args.workload),
                      "algorithmic_bytes_per_launch": total_bytes / len(bufs)},
         "layer_us_alone": layer_us,
+        "derived": derived_rates(layers, ms, world),
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms,
                 "how": "per step one copy of every layer's x from pinned host memory, the layers, one copy of every y "
@@ -489,8 +527,7 @@ def main():
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and args.cpu_budget > 0:
-        v, cores, desc = oracle_sample_run(layers, args.cpu_budget)
-        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+        line["cpu_baseline"] = cpu_baseline(layers, args.cpu_budget)
     if graph is not None:
         del graph
     if rank == 0:

@@ -70,3 +70,17 @@ def test_measured_traffic_needs_a_matching_hash(tmp_path, monkeypatch):
     prof.write_text("traffic_bytes_per_launch: 1234\nkernel_source_hash: 0000000000000000\n")
     assert bench.measured_traffic("w") is None
     assert bench.measured_traffic("missing") is None
+
+
+def test_derived_bf16_equivalent_rate():
+    layers = [("a", "int4", 32, 4096, 1024, 1), ("b", "fp6", 0, 2048, 512, 1)]
+    d = bench.derived_rates(layers, ms=0.5, world=2)
+    assert d["bf16_equivalent_gbps"] == pytest.approx(2 * (2 * 4096 * 1024 + 2 * 2048 * 512) / 0.5e-3 / 1e9)
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    layers = bench.workload_layers("int8-4096-m1")
+    cb = bench.cpu_baseline(layers, 0.2)
+    assert cb["kind"] == "oracle" and cb["unit"] == "GB/s" and cb["value"] > 0 and cb["cores"] >= 1
+    assert cb["cpu_model"] and cb["affinity_cores"] >= 1
+    assert cb["single_thread"]["cores"] == 1 and cb["single_thread"]["value"] > 0
